@@ -1,0 +1,20 @@
+"""Float64 CPU oracle for the bidirectional Video Delta Attention branch.
+
+Test infrastructure only: imported by tests/, by the smoke check and by the
+CPU-baseline leg of bench.py, never by the product path.
+"""
+from .vda_ref import (  # noqa: F401
+    RMS_EPS,
+    batch_rule_update,
+    boundary_states,
+    frame_stats,
+    frame_update,
+    gathered_state,
+    num_chunks,
+    rms_gate,
+    text_state,
+    vda_forward,
+    vda_forward_head,
+    vda_forward_head_naive,
+    window_bounds,
+)
