@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Benchmark of the bidirectional VDA branch on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one `vda_forward` call over the full-scale workload shaped like the
+paper's 14.3 s, 768p setting (B=1, H=48, T=60 interior latent frames,
+U=1008 tokens per frame, d_k=d_v=128, chunk 5, window +-1 chunk, bf16 I/O,
+fp32 states, text initial state from 256 prompt tokens).  Inputs are
+synthetic and seeded; they are resident in HBM when the timed region starts
+and far larger than L2 (about 3 GB read per step), so no L2 flush is needed.
+
+Metric: frame-tokens/s = B*T*U / time per step (every head, both scans, the
+readout and its epilogue).  With N GPUs (torchrun) every rank runs its own
+problem of the same size (weak scaling, no collective on the data path) and
+`value` = tokens of all ranks / max-over-ranks time.
+
+Prints ONE JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from frame_wise_delta_vda_b200 import inputs as gen  # noqa: E402
+
+WORKLOAD = "full"
+METRIC = "VDA fwd+rev frame-tokens/s at H=48,U=1008,d=128; % of HBM/tensor roofline"
+UNIT = "frame-tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv") \
+            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/vda_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "frame_wise_delta_vda_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
+    None when absent or taken on a different version of the kernel source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    if d.get("source_hash") != source_hash(*d.get("sources", [])):
+        return None
+    return d.get("bytes_per_launch_full")
+
+
+# ----------------------------------------------------------------------------
+def algorithmic(wl, tc):
+    """Per-stage algorithmic bytes and flops per launch for the workload (the
+    minimal in + out traffic of each kernel at its boundary; workspace
+    tensors A/M, B and the boundary states are fp32)."""
+    FH, U, d, e = wl.frame_heads, wl.U, wl.d, 2 if wl.dtype == "bf16" else 4
+    BH, NC = wl.B * wl.H, (wl.T + wl.chunk - 1) // wl.chunk
+    dd4 = d * d * 4
+    return {
+        "stats": {"bytes": FH * (2 * U * d * e + 4 * U + 2 * dd4), "flops": FH * 4 * U * d * d},
+        "inverse": {"bytes": FH * 2 * dd4, "flops": FH * d ** 3},
+        "scan": {"bytes": 2 * FH * 2 * dd4 + 2 * BH * (NC + 1) * dd4, "flops": 2 * FH * 2 * d ** 3},
+        "readout": {"bytes": FH * 3 * U * d * e + BH * NC * 2 * dd4 + 4 * d, "flops": FH * 2 * U * d * d},
+        "op": {"bytes": FH * (5 * U * d * e + 4 * U), "flops": FH * (6 * U * d * d + 5 * d ** 3)},
+    }
+
+
+STAGE_BOUND = {"stats": "hbm", "inverse": "alu", "scan": "hbm", "readout": "hbm"}
+STAGE_KERNEL = {"stats": ("k_stats", ["kernels_simt.cuh", "kernels_tc.cuh"]),
+                "inverse": ("k_gj_inverse", ["kernels_simt.cuh"]),
+                "scan": ("k_scan", ["kernels_simt.cuh", "kernels_tc.cuh"]),
+                "readout": ("k_readout", ["kernels_simt.cuh", "kernels_tc.cuh"])}
+
+
+def fp32_alu_peak_tflops(sm_mhz):
+    # 148 SMs x 128 FP32 lanes x 2 flops (FMA) per clock
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+# ----------------------------------------------------------------------------
+def cpu_baseline(wl, budget_s=15.0):
+    """The float64 oracle, as it stands, on this host's cores: whole heads of
+    the same workload until about `budget_s` seconds have been spent."""
+    import oracle as ref
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    heads, t_total = 0, 0.0
+    h = 0
+    while t_total < budget_s and h < wl.H:
+        x = gen.head_inputs(wl, 0, h)
+        w = gen.rms_weight(wl)
+        t0 = time.perf_counter()
+        S0 = ref.text_state(gen.as_f64(x["k_text"]), gen.as_f64(x["v_text"]), x["beta_text"]) \
+            if wl.text_tokens else None
+        ref.vda_forward_head(gen.as_f64(x["q"]), gen.as_f64(x["k"]), gen.as_f64(x["v"]), x["beta"],
+                             gen.as_f64(x["gate"]), w, S0, S0, wl.chunk, wl.window_chunks)
+        t_total += time.perf_counter() - t0
+        heads += 1
+        h += 1
+    value = wl.T * wl.U * heads / wl.H / t_total
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{heads} of {wl.H} heads of the {wl.name} workload (B=1, T={wl.T}, U={wl.U}, "
+                      f"d={wl.d}), fp64 NumPy, {t_total:.1f} s; value scaled to all heads"}
+
+
+def run_reference(args):
+    """The oracle arm: rank 0 times the fp64 oracle on one head per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle as ref
+    wl = gen.WORKLOADS[WORKLOAD]
+    x = gen.head_inputs(wl, 0, 0)
+    w = gen.rms_weight(wl)
+    args_f64 = [gen.as_f64(x["q"]), gen.as_f64(x["k"]), gen.as_f64(x["v"]), x["beta"], gen.as_f64(x["gate"])]
+    S0 = ref.text_state(gen.as_f64(x["k_text"]), gen.as_f64(x["v_text"]), x["beta_text"])
+
+    def step():
+        ref.vda_forward_head(*args_f64, w, S0, S0, wl.chunk, wl.window_chunks)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    value = wl.T * wl.U / wl.H / dt
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} T={wl.T} U={wl.U} d={wl.d} "
+                                   f"chunk={wl.chunk} window=+-{wl.window_chunks}",
+                       "sample": "one head of 48 per step (oracle, host cores)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "one head of the full workload per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+
+    from frame_wise_delta_vda_b200 import api
+    from frame_wise_delta_vda_b200._lib import lib
+    lib()  # fail loudly without the CUDA library
+
+    base = gen.WORKLOADS[WORKLOAD]
+    # every rank runs its own problem of the same size (weak scaling)
+    wl = gen.Workload(**{**base.__dict__, "seed": base.seed + 1000 * rank})
+
+    x = gen.make_inputs(wl)
+
+    def dev_t(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    t = {k: dev_t(v) for k, v in x.items()}
+    S0 = api.vda_text_state(t["k_text"], t["v_text"], t["beta_text"])
+    out = torch.empty_like(t["q"])
+    ws = api.workspace_for(t["q"], t["v"], wl.chunk)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        api.vda_forward(t["q"], t["k"], t["v"], t["beta"], t["gate"], t["rms_weight"], S0, S0,
+                        chunk=wl.chunk, window_chunks=wl.window_chunks, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert api.vda_device_status() == 0
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    timer = api.StageTimer(args.steps)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    stage_ms, calls = timer.read()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    status = api.vda_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    launches = api.vda_launches_per_forward(wl.B, wl.H, wl.T, wl.U, wl.d, wl.d, wl.chunk) * args.steps
+
+    # ---- end to end through the host-buffer entry point ------------------------
+    e2e_steps = args.e2e_steps if args.e2e_steps is not None else max(3, min(args.steps, 10))
+    host = {k: torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).pin_memory()
+            for k, v in x.items() if k in ("q", "k", "v", "gate", "beta", "rms_weight")}
+    for k in ("q", "k", "v", "gate"):
+        host[k] = host[k].view(torch.bfloat16)
+    S0_host = S0.cpu().pin_memory()
+    out_host = torch.empty_like(host["q"]).pin_memory()
+    hbuf = torch.empty(api.vda_forward_host_bytes(host["q"], host["v"], wl.chunk), dtype=torch.uint8, device=dev)
+
+    def e2e_step():
+        api.vda_forward_host(host["q"], host["k"], host["v"], host["beta"], host["gate"], host["rms_weight"],
+                             S0_host, S0_host, out_host, wl.chunk, wl.window_chunks, hbuf)
+
+    e2e_step()
+    if not torch.equal(out_host.view(torch.int16), out.cpu().view(torch.int16)):
+        raise RuntimeError("host-buffer path disagrees with the device path")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_s = (time.perf_counter() - t0) / e2e_steps
+    e2e_t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_s = float(e2e_t.item())
+    h2d = sum(int(host[k].numel() * host[k].element_size()) for k in host) + 2 * S0_host.numel() * 4
+    d2h = int(out_host.numel() * out_host.element_size())
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    # ---- roofline of the dominant kernel ------------------------------------
+    peaks, peak_src = load_peaks()
+    tc = api.vda_launches_per_forward(1, 1, 1, 1, 128, 128, 1) != 4 or False
+    alg = algorithmic(wl, tc)
+    dom = max(stage_ms, key=stage_ms.get)
+    dom_ms = stage_ms[dom] / max(calls, 1)
+    bound = STAGE_BOUND[dom]
+    sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    if bound == "hbm":
+        achieved = alg[dom]["bytes"] / (dom_ms * 1e-3) / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+        peak_note = f"hbm_gbs ({peak_src})"
+    else:
+        achieved = alg[dom]["flops"] / (dom_ms * 1e-3) / 1e12
+        peak, unit = fp32_alu_peak_tflops(sm_mhz), "TFLOP/s"
+        peak_note = f"FP32 FMA peak 148 SMs x 128 lanes x 2 at the sampled {sm_mhz:.0f} MHz"
+    kname, ksrc = STAGE_KERNEL[dom]
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": recorded_traffic(kname), "kernel": kname, "stage": dom,
+                "kernel_ms": dom_ms, "algorithmic_per_launch": alg[dom]["bytes" if bound == "hbm" else "flops"],
+                "peak_source": peak_note}
+    t_roof = max(alg["op"]["bytes"] / (peaks["hbm_gbs"] * 1e9),
+                 alg["op"]["flops"] / (peaks["bf16_tflops"] * 1e12))
+
+    tokens = wl.tokens * world
+    line = {
+        "metric": METRIC, "value": tokens / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} T={wl.T} U={wl.U} d={wl.d} chunk={wl.chunk} "
+                               f"window=+-{wl.window_chunks}, text S0 from 256 prompt tokens",
+                   "per_rank_problem": "independent problem of the same size per GPU",
+                   "l2": "inputs larger than L2 (about 3 GB read per step), no flush",
+                   "parallelism": f"replicas{world}"},
+        "roofline": roofline,
+        "op_roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof / (ms_max * 1e-3),
+                        "bytes": alg["op"]["bytes"], "flops": alg["op"]["flops"]},
+        "stage_ms": {k: v / max(calls, 1) for k, v in stage_ms.items()},
+        "clocks": clocks,
+        "e2e": {"value": tokens / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_s * 1e3, "api": "vda_forward_host (pinned host buffers)"},
+        "gpu_launches": launches,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

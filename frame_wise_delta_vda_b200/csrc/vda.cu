@@ -1,0 +1,525 @@
+// vda.cu - C ABI of the bidirectional Video Delta Attention branch (see
+// include/vda.h for the contract).  Validates arguments, plans the device
+// workspace and enqueues the kernels on the caller's stream.
+//
+// Paper: "Video DeltaNet" (arXiv 2609.20744), Algorithm 1 steps 3-7:
+//   stats (Eq. 3b) -> M_t = (I + A_t)^{-1} (Eq. 5, Appendix A.1) ->
+//   forward + reverse scans (Section 2.2) -> boundary gather (Appendix A.3,
+//   Eq. A.4) -> readout, RMSNorm, sigmoid gate (Eq. 1a, 1c).
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "vda.h"
+#include "common.cuh"
+#include "kernels_simt.cuh"
+#include "kernels_tc.cuh"
+
+namespace {
+
+using vda::ReadoutSimtCfg;
+
+constexpr size_t kAlign = 256;
+constexpr int kStages = 4;  // stats, inverse, scan, readout
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Plan {
+  int B, H, T, U, d, chunk, window, NC, dtype;
+  size_t BH, FH;
+  bool tc;               // tensor-core (tcgen05) kernels
+  size_t off_AM, off_B, off_states, total;
+};
+
+int check_sizes(int B, int H, int T, int U, int d_k, int d_v, int chunk, int window, int dtype) {
+  if (B < 1 || H < 1 || T < 1 || U < 1 || d_k < 1 || d_v < 1 || chunk < 1 || window < 0)
+    return VDA_ERR_INVALID_ARGUMENT;
+  if (dtype != VDA_BF16 && dtype != VDA_F32) return VDA_ERR_INVALID_ARGUMENT;
+  if (d_k != d_v) return VDA_ERR_UNSUPPORTED;
+  if (d_k != 16 && d_k != 32 && d_k != 64 && d_k != 128) return VDA_ERR_UNSUPPORTED;
+  // element counts must stay well inside 63 bits and grid limits
+  const double elems = (double)B * H * T * U * d_k;
+  if (elems > 4.0e12) return VDA_ERR_UNSUPPORTED;
+  if ((double)B * H * T > 2.0e9) return VDA_ERR_UNSUPPORTED;
+  return VDA_OK;
+}
+
+Plan make_plan(int B, int H, int T, int U, int d, int chunk, int window, int dtype) {
+  Plan p{};
+  p.B = B; p.H = H; p.T = T; p.U = U; p.d = d; p.chunk = chunk; p.window = window;
+  p.dtype = dtype;
+  p.NC = (T + chunk - 1) / chunk;
+  p.BH = (size_t)B * H;
+  p.FH = p.BH * T;
+  p.tc = vda::tc_path_supported(d, dtype);
+  const size_t dd = (size_t)d * d * sizeof(float);
+  size_t off = 0;
+  p.off_AM = off;     off = align_up(off + p.FH * dd);
+  p.off_B = off;      off = align_up(off + p.FH * dd);
+  p.off_states = off; off = align_up(off + 2 * p.BH * (size_t)(p.NC + 1) * dd);
+  p.total = off + vda::tc_extra_workspace_bytes(p.tc, p.FH, d);
+  return p;
+}
+
+// ----------------------------------------------------------------------------
+// per-stage timing (vda_timing_enable / vda_timing_read)
+struct Timing {
+  std::mutex mu;
+  int max_calls = 0;
+  int calls = 0;
+  std::vector<cudaEvent_t> ev;  // (kStages + 1) per call
+} g_timing;
+
+void timing_mark(int call_slot, int stage, cudaStream_t s) {
+  if (call_slot < 0) return;
+  cudaEventRecord(g_timing.ev[(size_t)call_slot * (kStages + 1) + stage], s);
+}
+
+int timing_begin_call() {
+  std::lock_guard<std::mutex> lk(g_timing.mu);
+  if (g_timing.max_calls <= 0 || g_timing.calls >= g_timing.max_calls) return -1;
+  return g_timing.calls++;
+}
+
+// ----------------------------------------------------------------------------
+template <int D, typename TIo>
+int launch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, int tslot,
+                float* stats_out) {
+  float* AM = reinterpret_cast<float*>(ws + p.off_AM);
+  float* Bm = reinterpret_cast<float*>(ws + p.off_B);
+  float* st = reinterpret_cast<float*>(ws + p.off_states);
+  const size_t fdd = p.FH * (size_t)D * D;
+
+  timing_mark(tslot, 0, s);
+  vda::k_stats_simt<D, TIo><<<(unsigned)p.FH, 256, 0, s>>>(
+      static_cast<const TIo*>(a.k), static_cast<const TIo*>(a.v), a.beta, p.U, AM, Bm);
+  if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  if (stats_out) {
+    if (cudaMemcpyAsync(stats_out, AM, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(stats_out + fdd, Bm, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return VDA_ERR_CUDA;
+  }
+  timing_mark(tslot, 1, s);
+  vda::k_gj_inverse<D><<<(unsigned)p.FH, 256, 0, s>>>(AM);
+  if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  if (stats_out) {
+    if (cudaMemcpyAsync(stats_out + 2 * fdd, AM, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return VDA_ERR_CUDA;
+  }
+  timing_mark(tslot, 2, s);
+  constexpr int RB = 16;
+  dim3 gs((unsigned)p.BH, 2, D / RB);
+  vda::k_scan_simt<D, RB><<<gs, D, 0, s>>>(AM, Bm, a.S0_fwd, a.S0_rev, st, (int)p.BH, p.T,
+                                           p.chunk, p.NC);
+  if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  timing_mark(tslot, 3, s);
+
+  using Cfg = ReadoutSimtCfg<D, TIo>;
+  const size_t smem = Cfg::smem_bytes();
+  if (cudaFuncSetAttribute(vda::k_readout_simt<D, TIo>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return VDA_ERR_CUDA;
+  const size_t pairs = p.BH * p.NC;
+  const long long tok_chunk = (long long)std::min(p.T, p.chunk) * p.U;
+  const long long per_cta = (long long)Cfg::WARPS * Cfg::TOK_PER_WARP * 4;
+  int splits = (int)std::min<long long>((tok_chunk + per_cta - 1) / per_cta,
+                                        std::max<long long>(1, 1184 / (long long)pairs));
+  splits = std::max(1, std::min(splits, 65535));
+  dim3 gr((unsigned)pairs, (unsigned)splits);
+  const float eps = a.eps > 0.f ? a.eps : 1e-6f;
+  vda::k_readout_simt<D, TIo><<<gr, 256, smem, s>>>(
+      static_cast<const TIo*>(a.q), static_cast<const TIo*>(a.gate), a.rms_weight, st,
+      static_cast<TIo*>(a.out), (int)p.BH, p.T, p.U, p.chunk, p.NC, p.window, eps);
+  if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  timing_mark(tslot, 4, s);
+  return VDA_OK;
+}
+
+template <typename TIo>
+int dispatch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, int tslot, float* so) {
+  switch (p.d) {
+    case 16: return launch_simt<16, TIo>(p, a, ws, s, tslot, so);
+    case 32: return launch_simt<32, TIo>(p, a, ws, s, tslot, so);
+    case 64: return launch_simt<64, TIo>(p, a, ws, s, tslot, so);
+    case 128: return launch_simt<128, TIo>(p, a, ws, s, tslot, so);
+  }
+  return VDA_ERR_UNSUPPORTED;
+}
+
+int validate_args(const vda_args* a) {
+  if (!a) return VDA_ERR_INVALID_ARGUMENT;
+  int rc = check_sizes(a->B, a->H, a->T, a->U, a->d_k, a->d_v, a->chunk, a->window_chunks, a->dtype);
+  if (rc != VDA_OK) return rc;
+  const void* req[] = {a->q, a->k, a->v, a->beta, a->gate, a->rms_weight, a->out};
+  for (const void* ptr : req)
+    if (!ptr || !aligned16(ptr)) return VDA_ERR_INVALID_ARGUMENT;
+  if ((a->S0_fwd && !aligned16(a->S0_fwd)) || (a->S0_rev && !aligned16(a->S0_rev)))
+    return VDA_ERR_INVALID_ARGUMENT;
+  return VDA_OK;
+}
+
+int forward_impl(const vda_args& a, char* ws, const Plan& p, float* states_out, float* stats_out) {
+  cudaStream_t s = static_cast<cudaStream_t>(a.stream);
+  const int tslot = timing_begin_call();
+  int rc;
+  if (p.tc) {
+    rc = vda::launch_tc(p.BH, p.T, p.U, p.chunk, p.NC, p.window, a, ws + p.off_AM, ws + p.off_B,
+                        ws + p.off_states, ws + p.total - vda::tc_extra_workspace_bytes(true, p.FH, p.d),
+                        s, stats_out,
+                        [&](int stage) { timing_mark(tslot, stage, s); });
+  } else if (p.dtype == VDA_BF16) {
+    rc = dispatch_simt<__nv_bfloat16>(p, a, ws, s, tslot, stats_out);
+  } else {
+    rc = dispatch_simt<float>(p, a, ws, s, tslot, stats_out);
+  }
+  if (rc != VDA_OK) return rc;
+  if (states_out) {
+    const size_t bytes = 2 * p.BH * (size_t)(p.NC + 1) * p.d * p.d * sizeof(float);
+    if (cudaMemcpyAsync(states_out, ws + p.off_states, bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return VDA_ERR_CUDA;
+  }
+  return VDA_OK;
+}
+
+int forward_alloc(const vda_args& a) {
+  int rc = validate_args(&a);
+  if (rc != VDA_OK) return rc;
+  const Plan p = make_plan(a.B, a.H, a.T, a.U, a.d_k, a.chunk, a.window_chunks, a.dtype);
+  cudaStream_t s = static_cast<cudaStream_t>(a.stream);
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, p.total, s) != cudaSuccess) return VDA_ERR_CUDA;
+  rc = forward_impl(a, static_cast<char*>(ws), p, nullptr, nullptr);
+  if (cudaFreeAsync(ws, s) != cudaSuccess && rc == VDA_OK) rc = VDA_ERR_CUDA;
+  return rc;
+}
+
+template <int D, typename TIo>
+int text_state_simt(const Plan& p, const void* k, const void* v, const float* beta, char* ws,
+                    cudaStream_t s) {
+  float* AM = reinterpret_cast<float*>(ws + p.off_AM);
+  float* Bm = reinterpret_cast<float*>(ws + p.off_B);
+  float* st = reinterpret_cast<float*>(ws + p.off_states);
+  vda::k_stats_simt<D, TIo><<<(unsigned)p.FH, 256, 0, s>>>(static_cast<const TIo*>(k),
+                                                           static_cast<const TIo*>(v), beta, p.U, AM, Bm);
+  if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  vda::k_gj_inverse<D><<<(unsigned)p.FH, 256, 0, s>>>(AM);
+  if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  dim3 gs((unsigned)p.BH, 1, D / 16);
+  vda::k_scan_simt<D, 16><<<gs, D, 0, s>>>(AM, Bm, nullptr, nullptr, st, (int)p.BH, 1, 1, p.NC);
+  if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  return VDA_OK;
+}
+
+template <typename TIo>
+int text_state_dispatch(const Plan& p, const void* k, const void* v, const float* beta, char* ws,
+                        cudaStream_t s) {
+  switch (p.d) {
+    case 16: return text_state_simt<16, TIo>(p, k, v, beta, ws, s);
+    case 32: return text_state_simt<32, TIo>(p, k, v, beta, ws, s);
+    case 64: return text_state_simt<64, TIo>(p, k, v, beta, ws, s);
+    case 128: return text_state_simt<128, TIo>(p, k, v, beta, ws, s);
+  }
+  return VDA_ERR_UNSUPPORTED;
+}
+
+int text_state_impl(const Plan& p, const void* k, const void* v, const float* beta, char* ws,
+                    cudaStream_t s) {
+  return p.dtype == VDA_BF16 ? text_state_dispatch<__nv_bfloat16>(p, k, v, beta, ws, s)
+                             : text_state_dispatch<float>(p, k, v, beta, ws, s);
+}
+
+// ----------------------------------------------------------------------------
+// host-buffer executor resources (one set per device)
+struct HostPipe {
+  bool init = false;
+  cudaStream_t h2d = nullptr, comp = nullptr, d2h = nullptr;
+  cudaEvent_t in_done[2], comp_done[2], out_done[2];
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[64];
+
+struct HostLayout {
+  int HG, groups;            // heads per group, number of groups
+  size_t in_elem;            // bytes per element of q/k/v/gate/out
+  size_t sz_qk, sz_v, sz_beta, sz_s0, sz_w;
+  size_t slot_off_q, slot_off_k, slot_off_v, slot_off_g, slot_off_beta, slot_off_s0f, slot_off_s0r,
+      slot_off_out, slot_off_ws, slot_bytes;
+  size_t ws_bytes;
+  size_t total;
+};
+
+HostLayout host_layout(int B, int H, int T, int U, int d, int chunk, int dtype) {
+  HostLayout L{};
+  const size_t BH = (size_t)B * H;
+  const int target_groups = 8;
+  L.HG = (int)std::max<size_t>(1, (BH + target_groups - 1) / target_groups);
+  L.groups = (int)((BH + L.HG - 1) / L.HG);
+  L.in_elem = dtype == VDA_BF16 ? 2 : 4;
+  const size_t tok = (size_t)L.HG * T * U;
+  L.sz_qk = tok * d * L.in_elem;
+  L.sz_v = L.sz_qk;
+  L.sz_beta = tok * sizeof(float);
+  L.sz_s0 = (size_t)L.HG * d * d * sizeof(float);
+  L.sz_w = (size_t)d * sizeof(float);
+  const Plan p = make_plan(1, L.HG, T, U, d, chunk, 0, dtype);
+  L.ws_bytes = p.total;
+  size_t off = 0;
+  L.slot_off_q = off;    off = align_up(off + L.sz_qk);
+  L.slot_off_k = off;    off = align_up(off + L.sz_qk);
+  L.slot_off_v = off;    off = align_up(off + L.sz_v);
+  L.slot_off_g = off;    off = align_up(off + L.sz_v);
+  L.slot_off_beta = off; off = align_up(off + L.sz_beta);
+  L.slot_off_s0f = off;  off = align_up(off + L.sz_s0);
+  L.slot_off_s0r = off;  off = align_up(off + L.sz_s0);
+  L.slot_off_out = off;  off = align_up(off + L.sz_v);
+  L.slot_off_ws = off;   off = align_up(off + L.ws_bytes);
+  L.slot_bytes = off;
+  L.total = align_up(L.sz_w) + 2 * L.slot_bytes;
+  return L;
+}
+
+}  // namespace
+
+// ============================================================================
+extern "C" {
+
+const char* vda_status_string(int status) {
+  switch (status) {
+    case VDA_OK: return "VDA_OK";
+    case VDA_ERR_INVALID_ARGUMENT: return "VDA_ERR_INVALID_ARGUMENT";
+    case VDA_ERR_UNSUPPORTED: return "VDA_ERR_UNSUPPORTED";
+    case VDA_ERR_WORKSPACE: return "VDA_ERR_WORKSPACE";
+    case VDA_ERR_CUDA: return "VDA_ERR_CUDA";
+    case VDA_ERR_TIMEOUT: return "VDA_ERR_TIMEOUT";
+  }
+  return "VDA_ERR_UNKNOWN";
+}
+
+size_t vda_workspace_bytes(int B, int H, int T, int U, int d_k, int d_v, int chunk, int dtype) {
+  if (check_sizes(B, H, T, U, d_k, d_v, chunk, 0, dtype) != VDA_OK) return 0;
+  return make_plan(B, H, T, U, d_k, chunk, 0, dtype).total;
+}
+
+int vda_launches_per_forward(int B, int H, int T, int U, int d_k, int d_v, int chunk, int dtype) {
+  if (check_sizes(B, H, T, U, d_k, d_v, chunk, 0, dtype) != VDA_OK) return 0;
+  const Plan p = make_plan(B, H, T, U, d_k, chunk, 0, dtype);
+  return p.tc ? vda::tc_launches_per_forward() : 4;
+}
+
+int vda_forward_ex(const vda_args* args, void* workspace, size_t workspace_bytes,
+                   float* states_out, float* stats_out) {
+  int rc = validate_args(args);
+  if (rc != VDA_OK) return rc;
+  if ((states_out && !aligned16(states_out)) || (stats_out && !aligned16(stats_out)))
+    return VDA_ERR_INVALID_ARGUMENT;
+  const Plan p = make_plan(args->B, args->H, args->T, args->U, args->d_k, args->chunk,
+                           args->window_chunks, args->dtype);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || workspace_bytes < p.total)
+    return VDA_ERR_WORKSPACE;
+  return forward_impl(*args, static_cast<char*>(workspace), p, states_out, stats_out);
+}
+
+int vda_forward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* beta,
+                const uint16_t* gate, const float* rms_weight, const float* S0_fwd,
+                const float* S0_rev, int B, int H, int T, int U, int d_k, int d_v, int chunk,
+                int window_chunks, uint16_t* out, void* stream) {
+  vda_args a{};
+  a.dtype = VDA_BF16;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.gate = gate; a.rms_weight = rms_weight;
+  a.S0_fwd = S0_fwd; a.S0_rev = S0_rev; a.out = out;
+  a.B = B; a.H = H; a.T = T; a.U = U; a.d_k = d_k; a.d_v = d_v;
+  a.chunk = chunk; a.window_chunks = window_chunks; a.eps = 1e-6f; a.stream = stream;
+  return forward_alloc(a);
+}
+
+int vda_forward_f32(const float* q, const float* k, const float* v, const float* beta,
+                    const float* gate, const float* rms_weight, const float* S0_fwd,
+                    const float* S0_rev, int B, int H, int T, int U, int d_k, int d_v, int chunk,
+                    int window_chunks, float* out, void* stream) {
+  vda_args a{};
+  a.dtype = VDA_F32;
+  a.q = q; a.k = k; a.v = v; a.beta = beta; a.gate = gate; a.rms_weight = rms_weight;
+  a.S0_fwd = S0_fwd; a.S0_rev = S0_rev; a.out = out;
+  a.B = B; a.H = H; a.T = T; a.U = U; a.d_k = d_k; a.d_v = d_v;
+  a.chunk = chunk; a.window_chunks = window_chunks; a.eps = 1e-6f; a.stream = stream;
+  return forward_alloc(a);
+}
+
+size_t vda_text_state_workspace_bytes(int B, int H, int L, int d_k, int d_v, int dtype) {
+  if (check_sizes(B, H, 1, L, d_k, d_v, 1, 0, dtype) != VDA_OK) return 0;
+  return make_plan(B, H, 1, L, d_k, 1, 0, dtype).total;
+}
+
+int vda_text_state(int dtype, const void* k_text, const void* v_text, const float* beta_text,
+                   int B, int H, int L, int d_k, int d_v, float* S_out, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, 1, L, d_k, d_v, 1, 0, dtype);
+  if (rc != VDA_OK) return rc;
+  if (!k_text || !v_text || !beta_text || !S_out || !aligned16(k_text) || !aligned16(v_text) ||
+      !aligned16(beta_text) || !aligned16(S_out))
+    return VDA_ERR_INVALID_ARGUMENT;
+  const Plan p = make_plan(B, H, 1, L, d_k, 1, 0, dtype);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || workspace_bytes < p.total)
+    return VDA_ERR_WORKSPACE;
+  // One frame of L tokens per (b, h): stats -> inverse -> one scan step from
+  // the zero state.  The readout is not needed, so only those three run.
+  rc = text_state_impl(p, k_text, v_text, beta_text, static_cast<char*>(workspace),
+                       static_cast<cudaStream_t>(stream));
+  if (rc != VDA_OK) return rc;
+  // forward state after the single frame sits at states[0][bh][1]
+  const size_t dd = (size_t)d_k * d_k * sizeof(float);
+  if (cudaMemcpy2DAsync(S_out, dd, static_cast<char*>(workspace) + p.off_states + dd, 2 * dd, dd,
+                        p.BH, cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return VDA_ERR_CUDA;
+  return VDA_OK;
+}
+
+size_t vda_forward_host_bytes(int B, int H, int T, int U, int d_k, int d_v, int chunk, int dtype) {
+  if (check_sizes(B, H, T, U, d_k, d_v, chunk, 0, dtype) != VDA_OK) return 0;
+  return host_layout(B, H, T, U, d_k, chunk, dtype).total;
+}
+
+int vda_forward_host(const vda_args* ha, void* device_buffer, size_t device_bytes) {
+  if (!ha) return VDA_ERR_INVALID_ARGUMENT;
+  int rc = check_sizes(ha->B, ha->H, ha->T, ha->U, ha->d_k, ha->d_v, ha->chunk, ha->window_chunks,
+                       ha->dtype);
+  if (rc != VDA_OK) return rc;
+  const void* req[] = {ha->q, ha->k, ha->v, ha->beta, ha->gate, ha->rms_weight, ha->out};
+  for (const void* ptr : req)
+    if (!ptr) return VDA_ERR_INVALID_ARGUMENT;
+  const HostLayout L = host_layout(ha->B, ha->H, ha->T, ha->U, ha->d_k, ha->chunk, ha->dtype);
+  if (!device_buffer || (reinterpret_cast<uintptr_t>(device_buffer) % kAlign) != 0 ||
+      device_bytes < L.total)
+    return VDA_ERR_WORKSPACE;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return VDA_ERR_CUDA;
+  HostPipe* P;
+  {
+    std::lock_guard<std::mutex> lk(g_pipe_mu);
+    P = &g_pipe[dev];
+    if (!P->init) {
+      bool ok = cudaStreamCreateWithFlags(&P->h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&P->comp, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&P->d2h, cudaStreamNonBlocking) == cudaSuccess;
+      for (int i = 0; ok && i < 2; ++i)
+        ok = cudaEventCreateWithFlags(&P->in_done[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&P->comp_done[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&P->out_done[i], cudaEventDisableTiming) == cudaSuccess;
+      if (!ok) return VDA_ERR_CUDA;
+      P->init = true;
+    }
+  }
+  char* base = static_cast<char*>(device_buffer);
+  float* d_w = reinterpret_cast<float*>(base);
+  char* slots = base + align_up(L.sz_w);
+  const size_t BH = (size_t)ha->B * ha->H;
+  const size_t per_head_tok = (size_t)ha->T * ha->U;
+  const int d = ha->d_k;
+#define VDA_CK(x) do { if ((x) != cudaSuccess) return VDA_ERR_CUDA; } while (0)
+  VDA_CK(cudaMemcpyAsync(d_w, ha->rms_weight, L.sz_w, cudaMemcpyHostToDevice, P->h2d));
+  for (int g = 0; g < L.groups; ++g) {
+    const int sl = g & 1;
+    char* S = slots + (size_t)sl * L.slot_bytes;
+    const size_t h0 = (size_t)g * L.HG;
+    const int nh = (int)std::min<size_t>(L.HG, BH - h0);
+    const size_t tokb = (size_t)nh * per_head_tok;
+    const size_t eb = tokb * d * L.in_elem;
+    const size_t off_e = h0 * per_head_tok * d * L.in_elem;
+    // the slot's inputs are free once group g-2 finished computing
+    if (g >= 2) VDA_CK(cudaStreamWaitEvent(P->h2d, P->comp_done[sl], 0));
+    VDA_CK(cudaMemcpyAsync(S + L.slot_off_q, static_cast<const char*>(ha->q) + off_e, eb, cudaMemcpyHostToDevice, P->h2d));
+    VDA_CK(cudaMemcpyAsync(S + L.slot_off_k, static_cast<const char*>(ha->k) + off_e, eb, cudaMemcpyHostToDevice, P->h2d));
+    VDA_CK(cudaMemcpyAsync(S + L.slot_off_v, static_cast<const char*>(ha->v) + off_e, eb, cudaMemcpyHostToDevice, P->h2d));
+    VDA_CK(cudaMemcpyAsync(S + L.slot_off_g, static_cast<const char*>(ha->gate) + off_e, eb, cudaMemcpyHostToDevice, P->h2d));
+    VDA_CK(cudaMemcpyAsync(S + L.slot_off_beta, ha->beta + h0 * per_head_tok, tokb * sizeof(float),
+                           cudaMemcpyHostToDevice, P->h2d));
+    const size_t s0b = (size_t)nh * d * d * sizeof(float);
+    if (ha->S0_fwd)
+      VDA_CK(cudaMemcpyAsync(S + L.slot_off_s0f, ha->S0_fwd + h0 * d * d, s0b, cudaMemcpyHostToDevice, P->h2d));
+    if (ha->S0_rev)
+      VDA_CK(cudaMemcpyAsync(S + L.slot_off_s0r, ha->S0_rev + h0 * d * d, s0b, cudaMemcpyHostToDevice, P->h2d));
+    VDA_CK(cudaEventRecord(P->in_done[sl], P->h2d));
+
+    VDA_CK(cudaStreamWaitEvent(P->comp, P->in_done[sl], 0));
+    if (g >= 2) VDA_CK(cudaStreamWaitEvent(P->comp, P->out_done[sl], 0));
+    vda_args a = *ha;
+    a.B = 1; a.H = nh;
+    a.q = S + L.slot_off_q; a.k = S + L.slot_off_k; a.v = S + L.slot_off_v; a.gate = S + L.slot_off_g;
+    a.beta = reinterpret_cast<const float*>(S + L.slot_off_beta);
+    a.rms_weight = d_w;
+    a.S0_fwd = ha->S0_fwd ? reinterpret_cast<const float*>(S + L.slot_off_s0f) : nullptr;
+    a.S0_rev = ha->S0_rev ? reinterpret_cast<const float*>(S + L.slot_off_s0r) : nullptr;
+    a.out = S + L.slot_off_out;
+    a.stream = P->comp;
+    const Plan p = make_plan(1, nh, a.T, a.U, d, a.chunk, a.window_chunks, a.dtype);
+    rc = forward_impl(a, S + L.slot_off_ws, p, nullptr, nullptr);
+    if (rc != VDA_OK) return rc;
+    VDA_CK(cudaEventRecord(P->comp_done[sl], P->comp));
+
+    VDA_CK(cudaStreamWaitEvent(P->d2h, P->comp_done[sl], 0));
+    VDA_CK(cudaMemcpyAsync(static_cast<char*>(ha->out) + off_e, S + L.slot_off_out, eb,
+                           cudaMemcpyDeviceToHost, P->d2h));
+    VDA_CK(cudaEventRecord(P->out_done[sl], P->d2h));
+  }
+  VDA_CK(cudaStreamSynchronize(P->d2h));
+  VDA_CK(cudaStreamSynchronize(P->comp));
+#undef VDA_CK
+  return VDA_OK;
+}
+
+int vda_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return VDA_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, vda::g_device_error, sizeof(word)) != cudaSuccess) return VDA_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemcpyToSymbol(vda::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return VDA_ERR_CUDA;
+    return VDA_ERR_TIMEOUT;
+  }
+  return VDA_OK;
+}
+
+int vda_timing_enable(int max_calls) {
+  std::lock_guard<std::mutex> lk(g_timing.mu);
+  for (cudaEvent_t e : g_timing.ev) cudaEventDestroy(e);
+  g_timing.ev.clear();
+  g_timing.calls = 0;
+  g_timing.max_calls = 0;
+  if (max_calls <= 0) return VDA_OK;
+  g_timing.ev.resize((size_t)max_calls * (kStages + 1));
+  for (auto& e : g_timing.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) return VDA_ERR_CUDA;
+  g_timing.max_calls = max_calls;
+  return VDA_OK;
+}
+
+int vda_timing_read(float* stage_ms, int n_stages, int* calls) {
+  std::lock_guard<std::mutex> lk(g_timing.mu);
+  if (!stage_ms || n_stages < 1) return VDA_ERR_INVALID_ARGUMENT;
+  for (int i = 0; i < n_stages; ++i) stage_ms[i] = 0.f;
+  const int n = g_timing.calls;
+  for (int c = 0; c < n; ++c) {
+    cudaEvent_t* e = &g_timing.ev[(size_t)c * (kStages + 1)];
+    if (cudaEventSynchronize(e[kStages]) != cudaSuccess) return VDA_ERR_CUDA;
+    for (int st = 0; st < std::min(n_stages, kStages); ++st) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, e[st], e[st + 1]) != cudaSuccess) return VDA_ERR_CUDA;
+      stage_ms[st] += ms;
+    }
+  }
+  if (calls) *calls = n;
+  for (cudaEvent_t e : g_timing.ev) cudaEventDestroy(e);
+  g_timing.ev.clear();
+  g_timing.calls = 0;
+  g_timing.max_calls = 0;
+  return VDA_OK;
+}
+
+}  // extern "C"

@@ -9,6 +9,8 @@ from .vda_ref import (  # noqa: F401
     boundary_states,
     frame_stats,
     frame_update,
+    forward_scan,
+    reverse_scan,
     gathered_state,
     num_chunks,
     rms_gate,

@@ -1,0 +1,49 @@
+"""Shared helpers for the test-suite: move generated inputs to torch, run the
+oracle per head, and compare with the relative Frobenius metric."""
+
+from __future__ import annotations
+
+import numpy as np
+
+import oracle as ref
+from frame_wise_delta_vda_b200 import inputs as gen
+
+# output tolerance per I/O dtype (relative Frobenius error per (b, h))
+TOL = {"bf16": 1e-2, "f32": 1e-4}
+# diagnostic bound for intermediates: 10x tighter than the output bound
+TOL_INTER = {"bf16": 1e-3, "f32": 1e-5}
+
+
+def to_torch(arr, device):
+    import torch
+    if arr.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(arr)).to(device)
+
+
+def to_numpy_f64(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        bits = t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        return gen.bf16_bits_to_f32(bits).astype(np.float64)
+    return t.detach().cpu().double().numpy()
+
+
+def rel_err(got, want):
+    n = np.linalg.norm(want)
+    d = np.linalg.norm(got - want)
+    if n == 0.0:
+        return 0.0 if d == 0.0 else np.inf
+    return d / n
+
+
+def oracle_head(x, wl, S0f=None, S0r=None, keep=False, w=None):
+    """Oracle output for one head's generated inputs (dict from head_inputs)."""
+    return ref.vda_forward_head(gen.as_f64(x["q"]), gen.as_f64(x["k"]), gen.as_f64(x["v"]),
+                                x["beta"], gen.as_f64(x["gate"]),
+                                gen.rms_weight(wl) if w is None else w,
+                                S0f, S0r, wl.chunk, wl.window_chunks, keep=keep)
+
+
+def oracle_text_state(x):
+    return ref.text_state(gen.as_f64(x["k_text"]), gen.as_f64(x["v_text"]), x["beta_text"])

@@ -1,0 +1,113 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the GPU."""
+
+import ctypes
+import re
+
+import pytest
+
+from frame_wise_delta_vda_b200 import _lib
+from frame_wise_delta_vda_b200._lib import VdaArgs
+
+
+@pytest.fixture(scope="module")
+def L():
+    return _lib.lib()
+
+
+def test_library_exports_every_header_symbol(L):
+    names = _lib.header_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(L, n), n
+    # and the binding declares every one of them
+    assert set(names) == set(_lib._SIGNATURES)
+
+
+def test_status_strings(L):
+    assert L.vda_status_string(0) == b"VDA_OK"
+    assert L.vda_status_string(1) == b"VDA_ERR_INVALID_ARGUMENT"
+    assert L.vda_status_string(5) == b"VDA_ERR_TIMEOUT"
+    assert L.vda_status_string(99) == b"VDA_ERR_UNKNOWN"
+
+
+def test_status_enum_matches_header():
+    text = open(_lib.HEADER).read()
+    for name in ("VDA_OK", "VDA_ERR_INVALID_ARGUMENT", "VDA_ERR_UNSUPPORTED", "VDA_ERR_WORKSPACE",
+                 "VDA_ERR_CUDA", "VDA_ERR_TIMEOUT", "VDA_BF16", "VDA_F32"):
+        m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
+        assert m and int(m.group(1)) == getattr(_lib, name), name
+
+
+def test_workspace_bytes(L):
+    # full-scale workload: A/M and B per frame-head plus chunk-boundary states
+    n = L.vda_workspace_bytes(1, 48, 60, 1008, 128, 128, 5, 0)
+    fh, dd = 48 * 60, 128 * 128 * 4
+    assert n >= 2 * fh * dd + 2 * 48 * 13 * dd
+    assert n % 256 == 0 or n > 0
+    assert L.vda_workspace_bytes(0, 48, 60, 1008, 128, 128, 5, 0) == 0
+    assert L.vda_workspace_bytes(1, 1, 1, 1, 128, 64, 5, 0) == 0      # d_k != d_v
+    assert L.vda_workspace_bytes(1, 1, 1, 1, 96, 96, 5, 0) == 0       # unsupported d
+    assert L.vda_workspace_bytes(1, 1, 1, 1, 16, 16, 5, 7) == 0       # bad dtype
+
+
+def _args(**kw):
+    a = VdaArgs()
+    a.dtype = 0
+    for f in ("q", "k", "v", "beta", "gate", "rms_weight", "out"):
+        setattr(a, f, 0x10000)          # aligned dummy addresses, never dereferenced
+    a.S0_fwd = None
+    a.S0_rev = None
+    a.B, a.H, a.T, a.U, a.d_k, a.d_v, a.chunk, a.window_chunks = 1, 2, 10, 16, 16, 16, 5, 1
+    a.eps = 1e-6
+    a.stream = None
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), 1), (dict(T=-1), 1), (dict(U=0), 1), (dict(chunk=0), 1), (dict(window_chunks=-1), 1),
+    (dict(q=None), 1), (dict(out=None), 1), (dict(beta=None), 1), (dict(rms_weight=None), 1),
+    (dict(k=0x10004), 1),                  # misaligned
+    (dict(S0_fwd=0x10008), 1),             # misaligned optional pointer
+    (dict(dtype=3), 1),
+    (dict(d_k=16, d_v=32), 2),             # d_k != d_v
+    (dict(d_k=48, d_v=48), 2),             # unsupported head dim
+])
+def test_forward_ex_rejects_bad_arguments(L, kw, status):
+    a = _args(**kw)
+    rc = L.vda_forward_ex(ctypes.byref(a), ctypes.c_void_p(0x100000), 1 << 30, None, None)
+    assert rc == status
+
+
+def test_forward_ex_rejects_small_or_misaligned_workspace(L):
+    a = _args()
+    need = L.vda_workspace_bytes(1, 2, 10, 16, 16, 16, 5, 0)
+    assert L.vda_forward_ex(ctypes.byref(a), None, need, None, None) == 3
+    assert L.vda_forward_ex(ctypes.byref(a), ctypes.c_void_p(0x100000), need - 1, None, None) == 3
+    assert L.vda_forward_ex(ctypes.byref(a), ctypes.c_void_p(0x100010), need, None, None) == 3
+    assert L.vda_forward_ex(None, ctypes.c_void_p(0x100000), need, None, None) == 1
+
+
+def test_text_state_and_host_entry_validation(L):
+    assert L.vda_text_state(0, None, None, None, 1, 1, 4, 16, 16, None, None, 0, None) == 1
+    assert L.vda_text_state(0, 0x100, 0x100, 0x100, 1, 1, 4, 16, 32, 0x100, None, 0, None) == 2
+    assert L.vda_text_state_workspace_bytes(1, 1, 4, 16, 16, 0) > 0
+    a = _args(q=None)
+    assert L.vda_forward_host(ctypes.byref(a), ctypes.c_void_p(0x100000), 1 << 30) == 1
+    a = _args()
+    assert L.vda_forward_host(ctypes.byref(a), ctypes.c_void_p(0x100000), 16) == 3
+    assert L.vda_forward_host_bytes(1, 48, 60, 1008, 128, 128, 5, 0) > 0
+
+
+def test_launch_count(L):
+    assert L.vda_launches_per_forward(1, 2, 10, 16, 16, 16, 5, 1) >= 4
+    assert L.vda_launches_per_forward(1, 2, 10, 16, 16, 24, 5, 1) == 0
+
+
+def test_timing_read_without_calls(L):
+    ms = (ctypes.c_float * 4)()
+    calls = ctypes.c_int(-1)
+    assert L.vda_timing_read(ms, 4, ctypes.byref(calls)) == 0
+    assert calls.value == 0 and list(ms) == [0.0] * 4
