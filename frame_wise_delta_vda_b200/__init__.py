@@ -6,11 +6,12 @@ Importing the package does not load the library, so the seeded input
 generator (``frame_wise_delta_vda_b200.inputs``) works on machines without it.
 """
 
+import importlib
+
 __all__ = ["api", "inputs"]
 
 
 def __getattr__(name):
-    if name == "api":
-        from . import api
-        return api
+    if name in ("api", "inputs", "build"):
+        return importlib.import_module(f".{name}", __name__)
     raise AttributeError(name)
