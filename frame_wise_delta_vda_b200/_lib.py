@@ -22,6 +22,7 @@ VDA_ERR_CUDA = 4
 VDA_ERR_TIMEOUT = 5
 VDA_BF16 = 0
 VDA_F32 = 1
+NOALLOC_SCRATCH_BYTES = 16 << 20   # VDA_NOALLOC_SCRATCH_BYTES in include/vda.h
 
 c_int, c_size_t, c_void_p, c_float = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
 c_float_p = ctypes.POINTER(ctypes.c_float)
@@ -51,6 +52,7 @@ _SIGNATURES = {
                        + [c_void_p, c_void_p, c_size_t, c_void_p]),
     "vda_forward_host_bytes": (c_size_t, [c_int] * 8),
     "vda_forward_host": (c_int, [ctypes.POINTER(VdaArgs), c_void_p, c_size_t]),
+    "vda_forward_noalloc": (c_int, [ctypes.POINTER(VdaArgs)]),
     "vda_device_status": (c_int, [c_void_p]),
     "vda_timing_enable": (c_int, [c_int]),
     "vda_timing_read": (c_int, [c_float_p, c_int, c_int_p]),

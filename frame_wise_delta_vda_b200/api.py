@@ -163,6 +163,19 @@ def vda_forward_host(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk
     return out
 
 
+def vda_forward_noalloc(q, k, v, beta, gate, rms_weight, S0_fwd=None, S0_rev=None, chunk=5,
+                        window_chunks=1, out=None, eps=1e-6, stream=None):
+    """Forward through `vda_forward_noalloc`: the library uses its fixed
+    internal scratch array instead of any allocation (sizes must fit in
+    NOALLOC_SCRATCH_BYTES of workspace).  `out` must be preallocated by callers
+    that cannot allocate; it is created here only as a convenience."""
+    if out is None:
+        out = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
+    a = make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks, eps, stream)
+    check(lib().vda_forward_noalloc(ctypes.byref(a)), "vda_forward_noalloc")
+    return out
+
+
 def vda_device_status(stream=None):
     """Synchronise and return the library's device error status (0 = OK)."""
     return int(lib().vda_device_status(_stream(stream)))

@@ -285,6 +285,33 @@ HostLayout host_layout(int B, int H, int T, int U, int d, int chunk, int dtype) 
   return L;
 }
 
+// ----------------------------------------------------------------------------
+// Scratch of vda_forward_noalloc: one fixed array in this module, so that the
+// entry point never allocates.  Its address is a device address only on the
+// device side; host code must obtain the device pointer with
+// cudaGetSymbolAddress (the symbol itself is a host-side stand-in).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[VDA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+int noalloc_scratch(char** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VDA_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return VDA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return VDA_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = static_cast<char*>(g_noalloc_ptr[dev]);
+  return VDA_OK;
+}
+
 }  // namespace
 
 // ============================================================================
@@ -473,6 +500,18 @@ int vda_forward_host(const vda_args* ha, void* device_buffer, size_t device_byte
   VDA_CK(cudaStreamSynchronize(P->comp));
 #undef VDA_CK
   return VDA_OK;
+}
+
+int vda_forward_noalloc(const vda_args* args) {
+  int rc = validate_args(args);
+  if (rc != VDA_OK) return rc;
+  const Plan p = make_plan(args->B, args->H, args->T, args->U, args->d_k, args->chunk,
+                           args->window_chunks, args->dtype);
+  if (p.total > VDA_NOALLOC_SCRATCH_BYTES) return VDA_ERR_WORKSPACE;
+  char* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc != VDA_OK) return rc;
+  return forward_impl(*args, scratch, p, nullptr, nullptr);
 }
 
 int vda_device_status(void* stream) {

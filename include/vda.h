@@ -149,6 +149,30 @@ VDA_API size_t vda_forward_host_bytes(int B, int H, int T, int U, int d_k, int d
                               int chunk, int dtype);
 VDA_API int vda_forward_host(const vda_args* host_args, void* device_buffer, size_t device_bytes);
 
+/* Forward without any allocation, for callers that cannot allocate device
+ * memory: host frameworks that own all device memory through their own
+ * allocator and have no way to hand this library a workspace, plugins loaded
+ * into such hosts, and fixed-footprint serving or real-time loops whose
+ * policy forbids allocator calls once they are running (a cudaMalloc there
+ * can block, fail under memory pressure, or synchronise the device).  Same
+ * arguments and result as vda_forward_ex with no workspace and no debug
+ * outputs; the scratch (statistics, transitions and chunk-boundary states)
+ * lives in one fixed array of VDA_NOALLOC_SCRATCH_BYTES inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ *   - Returns VDA_ERR_WORKSPACE when the sizes need more scratch than that
+ *     (vda_workspace_bytes() > VDA_NOALLOC_SCRATCH_BYTES); nothing is launched.
+ *   - The first call on each device looks up the array's device address with
+ *     the CUDA runtime (no allocation); make that first call before any stream
+ *     capture begins.
+ *   - Calls share the one array: two calls whose work overlaps on the GPU
+ *     (different streams, or different host threads, without ordering between
+ *     them) race and corrupt each other's results.  Every scratch word is
+ *     written before it is read in each call, so nothing left by an earlier
+ *     call leaks into a later one.
+ * The paper has no counterpart to this entry point; it is a deployment aid. */
+#define VDA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+VDA_API int vda_forward_noalloc(const vda_args* args);
+
 /* Synchronises `stream`, then reads and clears the library's device error
  * word for the current device: returns VDA_ERR_TIMEOUT if a kernel gave up a
  * bounded wait since the last call, VDA_ERR_CUDA on a CUDA error, else VDA_OK. */
