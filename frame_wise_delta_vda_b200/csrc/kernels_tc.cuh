@@ -1,20 +1,972 @@
-// kernels_tc.cuh - tcgen05 / TMA tensor-core kernels of the VDA path (d = 128,
-// bf16 I/O).  Not yet enabled: every size runs on the SIMT kernels.
+// kernels_tc.cuh - sm_100a tensor-core kernels of the VDA path for d = 128
+// with bf16 I/O: TMA-fed tcgen05 MMAs accumulating in TMEM.
+//
+// Paper: "Video DeltaNet" (arXiv 2609.20744).
+//   k_stats_tc    Eq. 3b: A_t = K^T Diag(beta) K, B_t = V^T Diag(beta) K
+//   k_gj_inverse  Eq. 5 / Appendix A.1: M_t = (I + A_t)^{-1}, written as the
+//                 bf16 hi/lo operand image the scan feeds to the tensor cores
+//   k_scan_tc     Section 2.2 + Eq. 5: S_t = (S_{t-1} + B_t) M_t, both
+//                 directions, fp32 state, 3-product bf16 hi/lo split MMAs
+//   k_readout_tc  Appendix A.3 (Eq. A.4) gather, Eq. 1a readout o = S~ q,
+//                 Eq. 1c RMSNorm + sigmoid gate, bf16 store
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstdlib>
+
 #include "common.cuh"
+#include "kernels_simt.cuh"
+#include "tc_ptx.cuh"
 #include "vda.h"
 
 namespace vda {
+namespace tc {
 
-inline bool tc_path_supported(int d, int dtype) { (void)d; (void)dtype; return false; }
-inline size_t tc_extra_workspace_bytes(bool tc, size_t FH, int d) { (void)tc; (void)FH; (void)d; return 0; }
+using namespace vda::ptx;
+
+constexpr int kD = 128;
+constexpr size_t kDD = (size_t)kD * kD;
+constexpr uint32_t kImgHalf = 32768;   // one bf16 128x128 operand image
+constexpr uint32_t kImgBytes = 65536;  // hi + lo images
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// ===========================================================================
+// k_stats_tc: per frame-head, with tokens on the MMA's K dimension,
+//   D[128 x 256] = (beta K)_hi^T [K | V]  +  [0 | (beta K)_lo^T V]
+// so D[:, 0:128] = A (bf16 beta*K) and D[:, 128:256] = B^T (beta*K split
+// into bf16 hi + lo: the B part carries ~16 significant bits, which the
+// correlated-key workload needs).  Both operands are MN-major: a TMA box of
+// 64 channels x 64 tokens lands as 64 rows of 128 B with the 128-B swizzle.
+//
+// Persistent CTAs (one per SM) walk frame-heads fh = blockIdx.x + i*grid.
+// Warps: 0-3 epilogue (TMEM -> global), 4-7 scale (beta*K hi/lo),
+//        8 TMA producer, 9 MMA issuer + TMEM owner.
+// Stage s holds K0 K1 V0 V1 (TMA), H0 H1 (hi), L0 L1 (lo): 8 x 8 KB.
+// TMEM: two 256-column accumulators (512 columns), so the epilogue of one
+// frame-head overlaps the MMAs of the next.
+// ===========================================================================
+struct StatsCfg {
+  static constexpr int UT = 64;
+  static constexpr int NST = 3;
+  static constexpr uint32_t BLK = UT * 128;          // 8192
+  static constexpr uint32_t OFF_KV = 0;
+  static constexpr uint32_t OFF_H = 4 * BLK;
+  static constexpr uint32_t OFF_L = 6 * BLK;
+  static constexpr uint32_t STAGE = 8 * BLK;         // 65536
+  static constexpr int THREADS = 320;
+  static constexpr uint32_t BAR_OFF = NST * STAGE;
+  static constexpr int NBAR = 3 * NST + 5;
+  static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
+};
+
+__global__ void __launch_bounds__(StatsCfg::THREADS, 1)
+k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+           const float* __restrict__ beta, int U, int FH,
+           float* __restrict__ A_out, float* __restrict__ B_out) {
+  using C = StatsCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
+  // barrier indices
+  const int FULL = 0, SCALED = C::NST, EMPTY = 2 * C::NST, TFULL = 3 * C::NST, TEMPTY = 3 * C::NST + 2,
+            DRAIN = 3 * C::NST + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(BAR(FULL + s), 1);
+      mbar_init(BAR(SCALED + s), 128);
+      mbar_init(BAR(EMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(BAR(TFULL + b), 1);
+      mbar_init(BAR(TEMPTY + b), 128);
+    }
+    mbar_init(BAR(DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nt = (U + C::UT - 1) / C::UT;
+  int last_it[C::NST];   // producer: last iteration issued on each stage
+  for (int s = 0; s < C::NST; ++s) last_it[s] = -1;
+
+  if (warp == 8) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int fh = blockIdx.x; ok && fh < FH; fh += gridDim.x) {
+        for (int tile = 0; tile < nt; ++tile, ++it) {
+          const uint32_t s = it % C::NST, ph = (it / C::NST) & 1u;
+          if (!mbar_wait(BAR(EMPTY + s), ph ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(BAR(FULL + s), 4 * C::BLK);
+          const uint32_t st = sbase + s * C::STAGE;
+          tma_load_3d(st + 0 * C::BLK, &tmK, 0, tile * C::UT, fh, BAR(FULL + s));
+          tma_load_3d(st + 1 * C::BLK, &tmK, 64, tile * C::UT, fh, BAR(FULL + s));
+          tma_load_3d(st + 2 * C::BLK, &tmV, 0, tile * C::UT, fh, BAR(FULL + s));
+          tma_load_3d(st + 3 * C::BLK, &tmV, 64, tile * C::UT, fh, BAR(FULL + s));
+          last_it[s] = (int)it;
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdN256 = idesc_bf16(128, 256, 1, 1);
+      constexpr uint32_t kIdN128 = idesc_bf16(128, 128, 1, 1);
+      uint32_t it = 0, lf = 0;
+      bool ok = true;
+      for (int fh = blockIdx.x; ok && fh < FH; fh += gridDim.x, ++lf) {
+        const uint32_t buf = lf & 1u, bph = (lf >> 1) & 1u;
+        if (!mbar_wait(BAR(TEMPTY + buf), bph ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * 256u;
+        for (int tile = 0; tile < nt; ++tile, ++it) {
+          const uint32_t s = it % C::NST, ph = (it / C::NST) & 1u;
+          if (!mbar_wait(BAR(SCALED + s), ph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = sbase + s * C::STAGE;
+#pragma unroll
+          for (int ks = 0; ks < C::UT / 16; ++ks) {
+            const uint32_t ko = (uint32_t)ks * 2048u;
+            mma_bf16_ss(d, desc_sw128(st + C::OFF_H + ko, C::BLK, 1024),
+                        desc_sw128(st + C::OFF_KV + ko, C::BLK, 1024), kIdN256, (tile | ks) != 0);
+            mma_bf16_ss(d + 128u, desc_sw128(st + C::OFF_L + ko, C::BLK, 1024),
+                        desc_sw128(st + C::OFF_KV + 2 * C::BLK + ko, C::BLK, 1024), kIdN128, 1u);
+          }
+          mma_commit(BAR(EMPTY + s));
+        }
+        if (!ok) break;
+        mma_commit(BAR(TFULL + buf));
+      }
+      // every issued MMA must finish before TMEM is released
+      mma_commit(BAR(DRAIN));
+      mbar_wait_drain(BAR(DRAIN), 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------- beta * K, split into bf16 hi + lo (same swizzled position)
+    const int st_id = tid - 128;
+    const int r = st_id & 63, hb = st_id >> 6;
+    auto beta_at = [&](int f, int tl) -> float {
+      const int u = tl * C::UT + r;
+      return (f < FH && u < U) ? __ldg(beta + (size_t)f * U + u) : 0.f;
+    };
+    uint32_t it = 0;
+    int fh = blockIdx.x, tile = 0;
+    float b_next = beta_at(fh, 0);
+    while (fh < FH) {
+      const float b = b_next;
+      int nfh = fh, ntile = tile + 1;
+      if (ntile == nt) { ntile = 0; nfh += gridDim.x; }
+      b_next = beta_at(nfh, ntile);
+      const uint32_t s = it % C::NST, ph = (it / C::NST) & 1u;
+      if (!mbar_wait(BAR(FULL + s), ph, abort_flag)) break;
+      uint8_t* stg = smem + s * C::STAGE;
+      const uint8_t* ksrc = stg + C::OFF_KV + hb * C::BLK + r * 128;
+      uint8_t* hdst = stg + C::OFF_H + hb * C::BLK + r * 128;
+      uint8_t* ldst = stg + C::OFF_L + hb * C::BLK + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int p = (c + r) & 7;   // rotate chunks across rows: conflict-free
+        const uint4 kv = *reinterpret_cast<const uint4*>(ksrc + p * 16);
+        const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float x0 = __uint_as_float(w[q] << 16) * b;
+          const float x1 = __uint_as_float(w[q] & 0xFFFF0000u) * b;
+          float h0, l0, h1, l1;
+          split_bf16(x0, h0, l0);
+          split_bf16(x1, h1, l1);
+          hw[q] = pack_bf16(h0, h1);
+          lw[q] = pack_bf16(l0, l1);
+        }
+        *reinterpret_cast<uint4*>(hdst + p * 16) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(ldst + p * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(SCALED + s));
+      ++it;
+      fh = nfh;
+      tile = ntile;
+    }
+  } else {
+    // ---------------- epilogue: TMEM lane i = channel i of D
+    const int i = warp * 32 + lane;
+    uint32_t lf = 0;
+    for (int fh = blockIdx.x; fh < FH; fh += gridDim.x, ++lf) {
+      const uint32_t buf = lf & 1u, bph = (lf >> 1) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(TFULL + buf), bph, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16) + buf * 256u;
+      float* Af = A_out + (size_t)fh * kDD;
+      float* Bf = B_out + (size_t)fh * kDD;
+#pragma unroll 1
+      for (int rr = 0; rr < 4; ++rr) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(trow + rr * 64, v0);
+        tmem_ld32(trow + rr * 64 + 32, v1);
+        tmem_wait_ld();
+        if (rr == 3) {
+          tc_fence_before();
+          mbar_arrive(BAR(TEMPTY + buf));
+        }
+        // D[i][col] -> A_out[col][i] (A is symmetric) / B_out[col - 128][i]
+        float* dst = rr < 2 ? Af + (size_t)(rr * 64) * kD : Bf + (size_t)((rr - 2) * 64) * kD;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          dst[(size_t)c * kD + i] = __uint_as_float(v0[c]);
+          dst[(size_t)(c + 32) * kD + i] = __uint_as_float(v1[c]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (warp == 8 && lane == 0 && *abort_flag) {  // let issued copies land before the CTA exits
+    for (int s = 0; s < C::NST; ++s)
+      if (last_it[s] >= 0) mbar_wait_drain(BAR(FULL + s), ((uint32_t)last_it[s] / C::NST) & 1u);
+  }
+}
+
+// ===========================================================================
+// Gauss-Jordan inverse (same elimination as k_gj_inverse in kernels_simt.cuh)
+// writing M = (I + A)^{-1} as the scan's tensor-core A operand: for the
+// product S_new[n][j] = sum_k X[n][k] M[k][j] the MMA computes
+// D[j][n] = sum_k M[k][j] X[n][k], i.e. operand element (j, k) = M[k][j],
+// MN-major (j contiguous) with the 128-B swizzle: two 64-column blocks of
+// 128 k-rows x 128 B.  M is stored split into bf16 hi (bytes [0, 32K)) and lo
+// (bytes [32K, 64K)); optionally M is also written as fp32 (debug output).
+// ===========================================================================
+__device__ __forceinline__ uint32_t mimg_offset(int j, int k) {
+  return (uint32_t)(j >> 6) * 16384u + sw128_offset((uint32_t)k, (uint32_t)(j & 63));
+}
+
+__global__ void __launch_bounds__(256)
+k_gj_inverse_img(const float* __restrict__ A, uint8_t* __restrict__ Mimg, float* __restrict__ M_f32) {
+  constexpr int D = kD, BS = 8;
+  __shared__ float s_row[2][D];
+  __shared__ float s_col[2][D];
+  const float* Ax = A + (size_t)blockIdx.x * kDD;
+  const int tid = threadIdx.x;
+  const int bi = tid >> 4, bj = tid & 15;
+  const int r0 = bi * BS, c0 = bj * BS;
+  float a[BS][BS];
+#pragma unroll
+  for (int i = 0; i < BS; ++i) {
+    const float4 x0 = *reinterpret_cast<const float4*>(Ax + (size_t)(r0 + i) * D + c0);
+    const float4 x1 = *reinterpret_cast<const float4*>(Ax + (size_t)(r0 + i) * D + c0 + 4);
+    a[i][0] = x0.x; a[i][1] = x0.y; a[i][2] = x0.z; a[i][3] = x0.w;
+    a[i][4] = x1.x; a[i][5] = x1.y; a[i][6] = x1.z; a[i][7] = x1.w;
+#pragma unroll
+    for (int j = 0; j < BS; ++j) a[i][j] += ((r0 + i) == (c0 + j)) ? 1.f : 0.f;
+  }
+  for (int kb = 0; kb < 16; ++kb) {
+#pragma unroll
+    for (int kk = 0; kk < BS; ++kk) {
+      const int k = kb * BS + kk;
+      const int buf = k & 1;
+      if (bi == kb) {
+#pragma unroll
+        for (int j = 0; j < BS; ++j) s_row[buf][c0 + j] = a[kk][j];
+      }
+      if (bj == kb) {
+#pragma unroll
+        for (int i = 0; i < BS; ++i) s_col[buf][r0 + i] = a[i][kk];
+      }
+      __syncthreads();
+      const float pinv = 1.0f / s_row[buf][k];
+      float c[BS], rs[BS];
+#pragma unroll
+      for (int i = 0; i < BS; ++i) c[i] = s_col[buf][r0 + i];
+#pragma unroll
+      for (int j = 0; j < BS; ++j) rs[j] = s_row[buf][c0 + j] * pinv;
+#pragma unroll
+      for (int i = 0; i < BS; ++i)
+#pragma unroll
+        for (int j = 0; j < BS; ++j) a[i][j] = fmaf(-c[i], rs[j], a[i][j]);
+      if (bi == kb) {
+#pragma unroll
+        for (int j = 0; j < BS; ++j) a[kk][j] = rs[j];
+      }
+      if (bj == kb) {
+#pragma unroll
+        for (int i = 0; i < BS; ++i) a[i][kk] = -c[i] * pinv;
+      }
+      if (bi == kb && bj == kb) a[kk][kk] = pinv;
+    }
+  }
+  // a[i][j] = M[r0 + i][c0 + j]: row index = k, column index = j of the operand
+  uint8_t* img = Mimg + (size_t)blockIdx.x * kImgBytes;
+#pragma unroll
+  for (int i = 0; i < BS; ++i) {
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float h0, l0, h1, l1;
+      split_bf16(a[i][2 * q], h0, l0);
+      split_bf16(a[i][2 * q + 1], h1, l1);
+      hw[q] = pack_bf16(h0, h1);
+      lw[q] = pack_bf16(l0, l1);
+    }
+    const uint32_t off = mimg_offset(c0, r0 + i);   // 8 consecutive j = one 16-B chunk
+    *reinterpret_cast<uint4*>(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(img + kImgHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+  if (M_f32) {
+    float* Mf = M_f32 + (size_t)blockIdx.x * kDD;
+#pragma unroll
+    for (int i = 0; i < BS; ++i) {
+      *reinterpret_cast<float4*>(Mf + (size_t)(r0 + i) * D + c0) = make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
+      *reinterpret_cast<float4*>(Mf + (size_t)(r0 + i) * D + c0 + 4) = make_float4(a[i][4], a[i][5], a[i][6], a[i][7]);
+    }
+  }
+}
+
+// ===========================================================================
+// k_scan_tc: one CTA per chain (b, h, direction); S in R^{128 x 128} fp32.
+// Step t: X = S + B_t (fp32), then S <- X M_t computed on the tensor cores as
+//   D[j][n] = sum_k M[k][j] X[n][k]  with  M = Mh + Ml,  X = Xh + Xl  (bf16)
+//   D = Mh Xh + Mh Xl + Ml Xh        (the dropped Ml Xl term is ~2^-16 rel.)
+// TMEM lane j holds column j of S (all 128 rows n in columns 0..127).
+// Warps 0-3: state (thread j = TMEM lane j): read S from TMEM, store boundary
+// states, add B_{t+1} (prefetched into registers), write the X hi/lo image
+// (K-major, 128-B swizzle).  Warp 4: bulk-copies the M image of the coming
+// steps (two stages).  Warp 5: MMA issuer, TMEM owner.
+// Boundary states: fwd[j] after frames [0, jC), rev[j] after [jC, T).
+// ===========================================================================
+struct ScanCfg {
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t OFF_M = 0;                    // 2 stages x 64 KB
+  static constexpr uint32_t OFF_X = 2 * kImgBytes;        // X hi (32 KB) + lo (32 KB)
+  static constexpr uint32_t BAR_OFF = 3 * kImgBytes;
+  static constexpr int NBAR = 2 + 2 + 1 + 1 + 1;           // mfull[2], mempty[2], xfull, dfull, drain
+  static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
+};
+
+__device__ __forceinline__ uint32_t ximg_offset(int n, int k) {
+  return (uint32_t)(k >> 6) * 16384u + sw128_offset((uint32_t)n, (uint32_t)(k & 63));
+}
+
+__global__ void __launch_bounds__(ScanCfg::THREADS, 1)
+k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
+          const float* __restrict__ S0f, const float* __restrict__ S0r,
+          float* __restrict__ states, int BH, int T, int chunk, int NC) {
+  using C = ScanCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
+  const int MFULL = 0, MEMPTY = 2, XFULL = 4, DFULL = 5, DRAIN = 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x, dir = blockIdx.y;
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(MFULL + s), 1);
+      mbar_init(BAR(MEMPTY + s), 1);
+    }
+    mbar_init(BAR(XFULL), 128);
+    mbar_init(BAR(DFULL), 1);
+    mbar_init(BAR(DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto frame_of = [&](int i) { return dir == 0 ? i : T - 1 - i; };
+  int last_i[2] = {-1, -1};   // producer: last step issued on each stage
+
+  if (warp == 4) {
+    // ---------------- M image producer
+    if (lane == 0) {
+      for (int i = 0; i < T; ++i) {
+        const uint32_t s = (uint32_t)i & 1u, ph = ((uint32_t)i >> 1) & 1u;
+        if (!mbar_wait(BAR(MEMPTY + s), ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(BAR(MFULL + s), kImgBytes);
+        const uint8_t* src = Mimg + ((size_t)bh * T + frame_of(i)) * kImgBytes;
+        const uint32_t dst = sbase + C::OFF_M + s * kImgBytes;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) bulk_load(dst + q * 16384u, src + q * 16384u, 16384u, BAR(MFULL + s));
+        last_i[s] = i;
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kId = idesc_bf16(128, 128, 1, 0);   // A (M image) MN-major, B (X) K-major
+      const uint32_t xh = sbase + C::OFF_X, xl = xh + kImgHalf;
+      for (int i = 0; i < T; ++i) {
+        const uint32_t s = (uint32_t)i & 1u, ph = ((uint32_t)i >> 1) & 1u;
+        if (!mbar_wait(BAR(XFULL), (uint32_t)i & 1u, abort_flag)) break;
+        if (!mbar_wait(BAR(MFULL + s), ph, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t mh = sbase + C::OFF_M + s * kImgBytes, ml = mh + kImgHalf;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t ao = (uint32_t)ks * 2048u;                              // 16 k-rows
+          const uint32_t bo = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;  // 16 k-columns
+          const uint64_t a_h = desc_sw128(mh + ao, 16384, 1024), a_l = desc_sw128(ml + ao, 16384, 1024);
+          const uint64_t b_h = desc_sw128(xh + bo, 16, 1024), b_l = desc_sw128(xl + bo, 16, 1024);
+          mma_bf16_ss(tmem, a_h, b_h, kId, ks != 0);
+          mma_bf16_ss(tmem, a_h, b_l, kId, 1u);
+          mma_bf16_ss(tmem, a_l, b_h, kId, 1u);
+        }
+        mma_commit(BAR(MEMPTY + s));
+        mma_commit(BAR(DFULL));
+      }
+      mma_commit(BAR(DRAIN));
+      mbar_wait_drain(BAR(DRAIN), 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- state warps: thread j owns column j of S
+    const int j = warp * 32 + lane;
+    const float* S0 = dir == 0 ? S0f : S0r;
+    float* st = states + ((size_t)dir * BH + bh) * (size_t)(NC + 1) * kDD;
+    uint8_t* xh = smem + C::OFF_X;
+    uint8_t* xl = xh + kImgHalf;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    float bnext[kD];
+
+    // initial state: store it as the first boundary, X_0 = S0 + B_{t0}
+    {
+      const int j0 = dir == 0 ? 0 : NC;
+      const float* B0 = Bm + ((size_t)bh * T + frame_of(0)) * kDD;
+#pragma unroll 8
+      for (int n = 0; n < kD; ++n) {
+        const float s0 = S0 ? __ldg(S0 + (size_t)bh * kDD + (size_t)n * kD + j) : 0.f;
+        st[(size_t)j0 * kDD + (size_t)n * kD + j] = s0;
+        float h, l;
+        split_bf16(s0 + __ldg(B0 + (size_t)n * kD + j), h, l);
+        const uint32_t off = ximg_offset(n, j);
+        *reinterpret_cast<__nv_bfloat16*>(xh + off) = __float2bfloat16_rn(h);
+        *reinterpret_cast<__nv_bfloat16*>(xl + off) = __float2bfloat16_rn(l);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(XFULL));
+    }
+    for (int i = 0; i < T; ++i) {
+      const bool more = i + 1 < T;
+      if (more) {
+        const float* Bn = Bm + ((size_t)bh * T + frame_of(i + 1)) * kDD;
+#pragma unroll
+        for (int n = 0; n < kD; ++n) bnext[n] = __ldg(Bn + (size_t)n * kD + j);
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(DFULL), (uint32_t)i & 1u, abort_flag))) break;
+      tc_fence_after();
+      const int t = frame_of(i);
+      int jb = -1;
+      if (dir == 0) {
+        if ((t + 1) % chunk == 0 || t == T - 1) jb = (t + chunk) / chunk;
+      } else if (t % chunk == 0) {
+        jb = t / chunk;
+      }
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        uint32_t v[32];
+        tmem_ld32(trow + cb * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int n = cb * 32 + c;
+          const float s = __uint_as_float(v[c]);
+          if (jb >= 0) st[(size_t)jb * kDD + (size_t)n * kD + j] = s;
+          if (more) {
+            float h, l;
+            split_bf16(s + bnext[n], h, l);
+            const uint32_t off = ximg_offset(n, j);
+            *reinterpret_cast<__nv_bfloat16*>(xh + off) = __float2bfloat16_rn(h);
+            *reinterpret_cast<__nv_bfloat16*>(xl + off) = __float2bfloat16_rn(l);
+          }
+        }
+      }
+      if (more) {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(XFULL));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+  if (warp == 4 && lane == 0 && *abort_flag) {  // let issued copies land before the CTA exits
+    for (int s = 0; s < 2; ++s)
+      if (last_i[s] >= 0) mbar_wait_drain(BAR(MFULL + s), ((uint32_t)last_i[s] >> 1) & 1u);
+  }
+}
+
+// ===========================================================================
+// k_readout_tc: out = sigmoid(g) * w * o / sqrt(mean(o^2) + eps), o = S~ q.
+// Work = 128-token tiles of each (b, h, chunk)'s contiguous token range; a
+// persistent CTA takes a contiguous run of tiles.  Per tile the MMA computes
+//   D[tok][i] = sum_k Q[tok][k] S~[i][k]     (S~ split into bf16 hi + lo)
+// with Q from TMA (K-major, 128-B swizzle) and the S~ image in shared memory,
+// built by the epilogue warps whenever the run enters a new (b, h, chunk):
+//   S~ = fwd[max(0, c - w)] + rev[min(NC, c + w + 1)]   (Appendix A.3)
+// TMEM lane = token row: RMSNorm is a per-thread sum of squares.  Gates come
+// through TMA as well; outputs are stored as 16-B vectors, rows past the
+// chunk end are skipped.
+// Warps 0-3: epilogue + S~ builder; warp 4: TMA producer; warp 5: MMA issuer.
+// ===========================================================================
+struct ReadoutCfg {
+  static constexpr int THREADS = 192;
+  static constexpr int TILE = 128;
+  static constexpr uint32_t TILE_BYTES = TILE * 256;           // 128 rows x 128 bf16
+  static constexpr uint32_t OFF_S = 0;                         // S~ hi (32 KB) + lo (32 KB)
+  static constexpr uint32_t OFF_Q = kImgBytes;                 // 2 x 32 KB
+  static constexpr uint32_t OFF_G = kImgBytes + 2 * TILE_BYTES; // 2 x 32 KB
+  static constexpr uint32_t OFF_W = kImgBytes + 4 * TILE_BYTES; // 128 floats
+  static constexpr uint32_t BAR_OFF = OFF_W + 512;
+  // qfull[2], qempty[2], gfull[2], gempty[2], tfull[2], tempty[2], sready, drain
+  static constexpr int NBAR = 14;
+  static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
+};
+
+struct ReadoutGeom {
+  int BH, T, U, chunk, NC, window;
+  int tpc;         // tiles of a full chunk
+  int tlast;       // tiles of the last chunk
+  int tph;         // tiles per head
+  long long total; // tiles over all heads
+};
+
+// tile index -> (bh, c, first row of the tile relative to the chunk, rows of the chunk)
+__device__ __forceinline__ void tile_coords(const ReadoutGeom& g, long long gt, int& bh, int& c, int& tr, int& rows) {
+  bh = (int)(gt / g.tph);
+  int rem = (int)(gt - (long long)bh * g.tph);
+  c = rem / g.tpc;
+  if (c > g.NC - 1) c = g.NC - 1;
+  tr = (rem - c * g.tpc) * ReadoutCfg::TILE;
+  const int f0 = c * g.chunk;
+  const int f1 = min(g.T, f0 + g.chunk);
+  rows = (f1 - f0) * g.U;
+}
+
+__global__ void __launch_bounds__(ReadoutCfg::THREADS, 1)
+k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
+             const float* __restrict__ w, const float* __restrict__ states,
+             __nv_bfloat16* __restrict__ out, ReadoutGeom g, float eps) {
+  using C = ReadoutCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
+  const int QFULL = 0, QEMPTY = 2, GFULL = 4, GEMPTY = 6, TFULL = 8, TEMPTY = 10, SREADY = 12, DRAIN = 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* sw = reinterpret_cast<float*>(smem + C::OFF_W);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // contiguous run of tiles of this CTA
+  const long long t_begin = g.total * blockIdx.x / gridDim.x;
+  const long long t_end = g.total * (blockIdx.x + 1) / gridDim.x;
+
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(QFULL + s), 1);
+      mbar_init(BAR(QEMPTY + s), 1);
+      mbar_init(BAR(GFULL + s), 1);
+      mbar_init(BAR(GEMPTY + s), 128);
+      mbar_init(BAR(TFULL + s), 1);
+      mbar_init(BAR(TEMPTY + s), 128);
+    }
+    mbar_init(BAR(SREADY), 128);
+    mbar_init(BAR(DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (tid < kD) sw[tid] = w[tid];
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const long long tokens_per_head = (long long)g.T * g.U;
+  int last_q[2] = {-1, -1}, last_g[2] = {-1, -1};   // producer: last tile issued per stage
+
+  if (warp == 4) {
+    // ---------------- TMA producer: Q and gate tiles
+    if (lane == 0) {
+      int k = 0;
+      for (long long gt = t_begin; gt < t_end; ++gt, ++k) {
+        int bh, c, tr, rows;
+        tile_coords(g, gt, bh, c, tr, rows);
+        const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.chunk * g.U + tr);
+        const uint32_t s = (uint32_t)k & 1u, ph = ((uint32_t)k >> 1) & 1u;
+        if (!mbar_wait(BAR(QEMPTY + s), ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(BAR(QFULL + s), C::TILE_BYTES);
+        const uint32_t qd = sbase + C::OFF_Q + s * C::TILE_BYTES;
+        tma_load_2d(qd, &tmQ, 0, row0, BAR(QFULL + s));
+        tma_load_2d(qd + C::TILE_BYTES / 2, &tmQ, 64, row0, BAR(QFULL + s));
+        last_q[s] = k;
+        if (!mbar_wait(BAR(GEMPTY + s), ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(BAR(GFULL + s), C::TILE_BYTES);
+        const uint32_t gd = sbase + C::OFF_G + s * C::TILE_BYTES;
+        tma_load_2d(gd, &tmG, 0, row0, BAR(GFULL + s));
+        tma_load_2d(gd + C::TILE_BYTES / 2, &tmG, 64, row0, BAR(GFULL + s));
+        last_g[s] = k;
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kId = idesc_bf16(128, 128, 0, 0);   // both K-major
+      const uint32_t sh = sbase + C::OFF_S, sl = sh + kImgHalf;
+      int k = 0, npair = 0, prev_bh = -1, prev_c = -1;
+      for (long long gt = t_begin; gt < t_end; ++gt, ++k) {
+        int bh, c, tr, rows;
+        tile_coords(g, gt, bh, c, tr, rows);
+        if (bh != prev_bh || c != prev_c) {
+          if (!mbar_wait(BAR(SREADY), (uint32_t)npair & 1u, abort_flag)) break;
+          ++npair;
+          prev_bh = bh;
+          prev_c = c;
+        }
+        const uint32_t s = (uint32_t)k & 1u, ph = ((uint32_t)k >> 1) & 1u;
+        if (!mbar_wait(BAR(QFULL + s), ph, abort_flag)) break;
+        if (!mbar_wait(BAR(TEMPTY + s), ph ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t q = sbase + C::OFF_Q + s * C::TILE_BYTES;
+        const uint32_t d = tmem + s * 128u;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t o = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
+          const uint64_t a = desc_sw128(q + o, 16, 1024);
+          mma_bf16_ss(d, a, desc_sw128(sh + o, 16, 1024), kId, ks != 0);
+          mma_bf16_ss(d, a, desc_sw128(sl + o, 16, 1024), kId, 1u);
+        }
+        mma_commit(BAR(QEMPTY + s));
+        mma_commit(BAR(TFULL + s));
+      }
+      mma_commit(BAR(DRAIN));
+      mbar_wait_drain(BAR(DRAIN), 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (thread r = token row r of the tile) + S~ builder
+    const int r = warp * 32 + lane;
+    const uint32_t trow_base = tmem + ((uint32_t)(warp * 32) << 16);
+    uint8_t* simg_h = smem + C::OFF_S;
+    uint8_t* simg_l = simg_h + kImgHalf;
+    int k = 0, prev_bh = -1, prev_c = -1;
+    const size_t sdir = (size_t)g.BH * (size_t)(g.NC + 1) * kDD;
+    for (long long gt = t_begin; gt < t_end; ++gt, ++k) {
+      int bh, c, tr, rows;
+      tile_coords(g, gt, bh, c, tr, rows);
+      if (bh != prev_bh || c != prev_c) {
+        // build S~ = fwd[max(0, c-w)] + rev[min(NC, c+w+1)]: thread r writes row i = r
+        const int jf = max(0, c - g.window), jr = min(g.NC, c + g.window + 1);
+        const float* Sf = states + (size_t)bh * (size_t)(g.NC + 1) * kDD + (size_t)jf * kDD + (size_t)r * kD;
+        const float* Sr = states + sdir + (size_t)bh * (size_t)(g.NC + 1) * kDD + (size_t)jr * kD * kD +
+                          (size_t)r * kD;
+#pragma unroll 4
+        for (int cc = 0; cc < 16; ++cc) {
+          const float4 f0 = __ldg(reinterpret_cast<const float4*>(Sf + cc * 8));
+          const float4 f1 = __ldg(reinterpret_cast<const float4*>(Sf + cc * 8 + 4));
+          const float4 r0v = __ldg(reinterpret_cast<const float4*>(Sr + cc * 8));
+          const float4 r1v = __ldg(reinterpret_cast<const float4*>(Sr + cc * 8 + 4));
+          const float x[8] = {f0.x + r0v.x, f0.y + r0v.y, f0.z + r0v.z, f0.w + r0v.w,
+                              f1.x + r1v.x, f1.y + r1v.y, f1.z + r1v.z, f1.w + r1v.w};
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float h0, l0, h1, l1;
+            split_bf16(x[2 * q], h0, l0);
+            split_bf16(x[2 * q + 1], h1, l1);
+            hw[q] = pack_bf16(h0, h1);
+            lw[q] = pack_bf16(l0, l1);
+          }
+          const uint32_t off = ximg_offset(r, cc * 8);   // row i = r, columns k = 8cc..8cc+7
+          *reinterpret_cast<uint4*>(simg_h + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(simg_l + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(BAR(SREADY));
+        prev_bh = bh;
+        prev_c = c;
+      }
+      const uint32_t s = (uint32_t)k & 1u, ph = ((uint32_t)k >> 1) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(TFULL + s), ph, abort_flag))) break;
+      tc_fence_after();
+      float o[kD];
+      const uint32_t trow = trow_base + s * 128u;
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        uint32_t v[32];
+        tmem_ld32(trow + cb * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) o[cb * 32 + c2] = __uint_as_float(v[c2]);
+      }
+      tc_fence_before();
+      mbar_arrive(BAR(TEMPTY + s));
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < kD; ++i) ss = fmaf(o[i], o[i], ss);
+      const float rinv = rsqrtf(ss * (1.0f / kD) + eps);
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(GFULL + s), ph, abort_flag))) break;
+      const uint8_t* gt_s = smem + C::OFF_G + s * C::TILE_BYTES;
+      const bool valid = tr + r < rows;
+      __nv_bfloat16* orow = out + ((size_t)bh * tokens_per_head + (size_t)c * g.chunk * g.U + tr + r) * kD;
+#pragma unroll
+      for (int cc = 0; cc < 16; ++cc) {
+        const uint32_t off = (uint32_t)(cc >> 3) * (C::TILE_BYTES / 2) + sw128_offset((uint32_t)r, (uint32_t)((cc & 7) * 8));
+        const uint4 gv = *reinterpret_cast<const uint4*>(gt_s + off);
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        uint32_t yw[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int i0 = cc * 8 + 2 * q;
+          const float g0 = __uint_as_float(gw[q] << 16), g1 = __uint_as_float(gw[q] & 0xFFFF0000u);
+          const float y0 = o[i0] * rinv * sw[i0] / (1.0f + __expf(-g0));
+          const float y1 = o[i0 + 1] * rinv * sw[i0 + 1] / (1.0f + __expf(-g1));
+          yw[q] = pack_bf16(y0, y1);
+        }
+        if (valid) *reinterpret_cast<uint4*>(orow + cc * 8) = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+      }
+      mbar_arrive(BAR(GEMPTY + s));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+  if (warp == 4 && lane == 0 && *abort_flag) {  // let issued copies land before the CTA exits
+    for (int s = 0; s < 2; ++s) {
+      if (last_q[s] >= 0) mbar_wait_drain(BAR(QFULL + s), ((uint32_t)last_q[s] >> 1) & 1u);
+      if (last_g[s] >= 0) mbar_wait_drain(BAR(GFULL + s), ((uint32_t)last_g[s] >> 1) & 1u);
+    }
+  }
+}
+
+// ===========================================================================
+// host side
+// ===========================================================================
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor [outer][mid][128] with a box of 64 x box_mid x 1, 128-B swizzle
+inline bool encode_bf16_3d(CUtensorMap* m, const void* base, uint64_t mid, uint64_t outer, uint32_t box_mid) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, mid, outer};
+  cuuint64_t strides[2] = {256, mid * 256};
+  cuuint32_t box[3] = {64, box_mid, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 matrix [rows][128] with a box of 64 x box_rows, 128-B swizzle
+inline bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {256};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// frame statistics for FH frame-heads of U tokens (K, V: [FH][U][128] bf16)
+inline int launch_stats(const void* K, const void* V, const float* beta, int U, size_t FH, float* A, float* B,
+                        cudaStream_t s) {
+  CUtensorMap tmK, tmV;
+  if (!encode_bf16_3d(&tmK, K, (uint64_t)U, FH, 64) || !encode_bf16_3d(&tmV, V, (uint64_t)U, FH, 64))
+    return VDA_ERR_CUDA;
+  if (cudaFuncSetAttribute(k_stats_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StatsCfg::SMEM) !=
+      cudaSuccess)
+    return VDA_ERR_CUDA;
+  const int grid = (int)std::min<size_t>(FH, (size_t)num_sms());
+  k_stats_tc<<<grid, StatsCfg::THREADS, StatsCfg::SMEM, s>>>(tmK, tmV, beta, U, (int)FH, A, B);
+  return cudaGetLastError() == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+}
+
+inline int launch_inverse_img(const float* A, uint8_t* Mimg, float* M_f32, size_t FH, cudaStream_t s) {
+  k_gj_inverse_img<<<(unsigned)FH, 256, 0, s>>>(A, Mimg, M_f32);
+  return cudaGetLastError() == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+}
+
+inline int launch_scan(const uint8_t* Mimg, const float* Bm, const float* S0f, const float* S0r, float* states,
+                       size_t BH, int T, int chunk, int NC, int ndir, cudaStream_t s) {
+  if (cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanCfg::SMEM) !=
+      cudaSuccess)
+    return VDA_ERR_CUDA;
+  dim3 grid((unsigned)BH, (unsigned)ndir);
+  k_scan_tc<<<grid, ScanCfg::THREADS, ScanCfg::SMEM, s>>>(Mimg, Bm, S0f, S0r, states, (int)BH, T, chunk, NC);
+  return cudaGetLastError() == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+}
+
+inline int launch_readout(const void* Q, const void* G, const float* w, const float* states, void* out,
+                          size_t BH, int T, int U, int chunk, int NC, int window, float eps, cudaStream_t s) {
+  ReadoutGeom g{};
+  g.BH = (int)BH; g.T = T; g.U = U; g.chunk = chunk; g.NC = NC; g.window = window;
+  const long long rows_full = (long long)std::min(T, chunk) * U;
+  const long long rows_last = (long long)(T - (NC - 1) * chunk) * U;
+  g.tpc = (int)((rows_full + ReadoutCfg::TILE - 1) / ReadoutCfg::TILE);
+  g.tlast = (int)((rows_last + ReadoutCfg::TILE - 1) / ReadoutCfg::TILE);
+  g.tph = (NC - 1) * g.tpc + g.tlast;
+  g.total = (long long)BH * g.tph;
+  const uint64_t rows = (uint64_t)BH * T * U;
+  CUtensorMap tmQ, tmG;
+  if (!encode_bf16_2d(&tmQ, Q, rows, ReadoutCfg::TILE) || !encode_bf16_2d(&tmG, G, rows, ReadoutCfg::TILE))
+    return VDA_ERR_CUDA;
+  if (cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ReadoutCfg::SMEM) !=
+      cudaSuccess)
+    return VDA_ERR_CUDA;
+  const int grid = (int)std::min<long long>(g.total, (long long)num_sms());
+  k_readout_tc<<<grid, ReadoutCfg::THREADS, ReadoutCfg::SMEM, s>>>(
+      tmQ, tmG, w, states, static_cast<__nv_bfloat16*>(out), g, eps);
+  return cudaGetLastError() == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+}
+
+}  // namespace tc
+
+// ---------------------------------------------------------------------------
+// path selection and the staged launch used by vda.cu
+inline bool tc_path_supported(int d, int dtype) { return d == 128 && dtype == VDA_BF16; }
+
+// extra workspace of the tensor-core path: the M hi/lo operand images
+inline size_t tc_extra_workspace_bytes(bool tc, size_t FH, int d) {
+  (void)d;
+  return tc ? FH * (size_t)tc::kImgBytes : 0;
+}
+
 inline int tc_launches_per_forward() { return 4; }
 
+// With VDA_DEBUG_SYNC=1 in the environment, every stage is followed by a
+// stream synchronisation and a check of the device error word, and a failing
+// stage is named on stderr (a debugging aid; off by default).
+inline bool debug_sync_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("VDA_DEBUG_SYNC");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+inline int debug_check(const char* stage, cudaStream_t s) {
+  if (!debug_sync_enabled()) return VDA_OK;
+  const cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "vda: stage %s failed: %s\n", stage, cudaGetErrorString(e));
+    return VDA_ERR_CUDA;
+  }
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) == cudaSuccess && word != 0) {
+    fprintf(stderr, "vda: stage %s gave up a bounded wait (device error word %u)\n", stage, word);
+    return VDA_ERR_TIMEOUT;
+  }
+  return VDA_OK;
+}
+
 template <typename MarkFn>
-int launch_tc(size_t, int, int, int, int, int, const vda_args&, char*, char*, char*, char*,
-              cudaStream_t, float*, MarkFn) {
-  return VDA_ERR_UNSUPPORTED;
+int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_args& a, char* ws_AM,
+              char* ws_B, char* ws_states, char* ws_img, cudaStream_t s, float* stats_out, MarkFn mark) {
+  const size_t FH = BH * (size_t)T;
+  const size_t fdd = FH * tc::kDD;
+  float* A = reinterpret_cast<float*>(ws_AM);
+  float* Bm = reinterpret_cast<float*>(ws_B);
+  float* st = reinterpret_cast<float*>(ws_states);
+  uint8_t* img = reinterpret_cast<uint8_t*>(ws_img);
+  int rc;
+  mark(0);
+  if ((rc = tc::launch_stats(a.k, a.v, a.beta, U, FH, A, Bm, s)) != VDA_OK) return rc;
+  if ((rc = debug_check("stats", s)) != VDA_OK) return rc;
+  if (stats_out) {
+    if (cudaMemcpyAsync(stats_out, A, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(stats_out + fdd, Bm, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return VDA_ERR_CUDA;
+  }
+  mark(1);
+  if ((rc = tc::launch_inverse_img(A, img, stats_out ? stats_out + 2 * fdd : nullptr, FH, s)) != VDA_OK) return rc;
+  if ((rc = debug_check("inverse", s)) != VDA_OK) return rc;
+  mark(2);
+  if ((rc = tc::launch_scan(img, Bm, a.S0_fwd, a.S0_rev, st, BH, T, chunk, NC, 2, s)) != VDA_OK) return rc;
+  if ((rc = debug_check("scan", s)) != VDA_OK) return rc;
+  mark(3);
+  const float eps = a.eps > 0.f ? a.eps : 1e-6f;
+  if ((rc = tc::launch_readout(a.q, a.gate, a.rms_weight, st, a.out, BH, T, U, chunk, NC, window, eps, s)) !=
+      VDA_OK)
+    return rc;
+  if ((rc = debug_check("readout", s)) != VDA_OK) return rc;
+  mark(4);
+  return VDA_OK;
+}
+
+// text state on the tensor-core kernels: stats over one frame of L tokens per
+// (b, h), inverse, one forward scan step from the zero state
+inline int tc_text_state(size_t BH, int L, const void* k, const void* v, const float* beta, char* ws_AM,
+                         char* ws_B, char* ws_states, char* ws_img, cudaStream_t s) {
+  float* A = reinterpret_cast<float*>(ws_AM);
+  float* Bm = reinterpret_cast<float*>(ws_B);
+  uint8_t* img = reinterpret_cast<uint8_t*>(ws_img);
+  int rc;
+  if ((rc = tc::launch_stats(k, v, beta, L, BH, A, Bm, s)) != VDA_OK) return rc;
+  if ((rc = tc::launch_inverse_img(A, img, nullptr, BH, s)) != VDA_OK) return rc;
+  return tc::launch_scan(img, Bm, nullptr, nullptr, reinterpret_cast<float*>(ws_states), BH, 1, 1, 1, 1, s);
 }
 
 }  // namespace vda

@@ -231,6 +231,9 @@ int text_state_dispatch(const Plan& p, const void* k, const void* v, const float
 
 int text_state_impl(const Plan& p, const void* k, const void* v, const float* beta, char* ws,
                     cudaStream_t s) {
+  if (p.tc)
+    return vda::tc_text_state(p.BH, p.U, k, v, beta, ws + p.off_AM, ws + p.off_B, ws + p.off_states,
+                              ws + p.total - vda::tc_extra_workspace_bytes(true, p.FH, p.d), s);
   return p.dtype == VDA_BF16 ? text_state_dispatch<__nv_bfloat16>(p, k, v, beta, ws, s)
                              : text_state_dispatch<float>(p, k, v, beta, ws, s);
 }
