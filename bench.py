@@ -49,7 +49,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="timed steps of the host-buffer (end-to-end) measurement; 0 skips it")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(gen.WORKLOADS),
+                    help="workload to run (the benchmark line is defined on 'full'; other "
+                         "workloads serve profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -136,7 +140,7 @@ def recorded_traffic(kernel):
 
 
 # ----------------------------------------------------------------------------
-def algorithmic(wl, tc):
+def algorithmic(wl):
     """Per-stage algorithmic bytes and flops per launch for the workload (the
     minimal in + out traffic of each kernel at its boundary; workspace
     tensors A/M, B and the boundary states are fp32)."""
@@ -258,19 +262,21 @@ def main():
     from frame_wise_delta_vda_b200._lib import lib
     lib()  # fail loudly without the CUDA library
 
-    base = gen.WORKLOADS[WORKLOAD]
+    base = gen.WORKLOADS[args.workload]
     # every rank runs its own problem of the same size (weak scaling)
     wl = gen.Workload(**{**base.__dict__, "seed": base.seed + 1000 * rank})
 
     x = gen.make_inputs(wl)
+    if "k_text" not in x:
+        x["k_text"], x["v_text"], x["beta_text"] = None, None, None
 
     def dev_t(a):
         if a.dtype == np.uint16:
             return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
         return torch.from_numpy(a).to(dev)
 
-    t = {k: dev_t(v) for k, v in x.items()}
-    S0 = api.vda_text_state(t["k_text"], t["v_text"], t["beta_text"])
+    t = {k: dev_t(v) for k, v in x.items() if v is not None}
+    S0 = api.vda_text_state(t["k_text"], t["v_text"], t["beta_text"]) if "k_text" in t else None
     out = torch.empty_like(t["q"])
     ws = api.workspace_for(t["q"], t["v"], wl.chunk)
     stream = torch.cuda.current_stream()
@@ -313,11 +319,26 @@ def main():
 
     # ---- end to end through the host-buffer entry point ------------------------
     e2e_steps = args.e2e_steps if args.e2e_steps is not None else max(3, min(args.steps, 10))
+    e2e = None
+    if e2e_steps > 0:
+        e2e = run_e2e(api, x, S0, out, wl, dev, e2e_steps, world, dist)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches)
+
+
+def run_e2e(api, x, S0, out, wl, dev, e2e_steps, world, dist):
+    """End-to-end timing through vda_forward_host with pinned host buffers."""
+    import torch
     host = {k: torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).pin_memory()
             for k, v in x.items() if k in ("q", "k", "v", "gate", "beta", "rms_weight")}
     for k in ("q", "k", "v", "gate"):
         host[k] = host[k].view(torch.bfloat16)
-    S0_host = S0.cpu().pin_memory()
+    S0_host = S0.cpu().pin_memory() if S0 is not None else None
     out_host = torch.empty_like(host["q"]).pin_memory()
     hbuf = torch.empty(api.vda_forward_host_bytes(host["q"], host["v"], wl.chunk), dtype=torch.uint8, device=dev)
 
@@ -340,19 +361,18 @@ def main():
     if world > 1:
         dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
     e2e_s = float(e2e_t.item())
-    h2d = sum(int(host[k].numel() * host[k].element_size()) for k in host) + 2 * S0_host.numel() * 4
+    h2d = sum(int(host[k].numel() * host[k].element_size()) for k in host)
+    if S0_host is not None:
+        h2d += 2 * S0_host.numel() * 4
     d2h = int(out_host.numel() * out_host.element_size())
+    return {"e2e_s": e2e_s, "h2d": h2d, "d2h": d2h}
 
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return
+
+def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches):
 
     # ---- roofline of the dominant kernel ------------------------------------
     peaks, peak_src = load_peaks()
-    tc = api.vda_launches_per_forward(1, 1, 1, 1, 128, 128, 1) != 4 or False
-    alg = algorithmic(wl, tc)
+    alg = algorithmic(wl)
     dom = max(stage_ms, key=stage_ms.get)
     dom_ms = stage_ms[dom] / max(calls, 1)
     bound = STAGE_BOUND[dom]
@@ -380,7 +400,8 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} T={wl.T} U={wl.U} d={wl.d} chunk={wl.chunk} "
-                               f"window=+-{wl.window_chunks}, text S0 from 256 prompt tokens",
+                               f"window=+-{wl.window_chunks}"
+                               + (f", text S0 from {wl.text_tokens} prompt tokens" if wl.text_tokens else ", S0 = 0"),
                    "per_rank_problem": "independent problem of the same size per GPU",
                    "l2": "inputs larger than L2 (about 3 GB read per step), no flush",
                    "parallelism": f"replicas{world}"},
@@ -389,8 +410,10 @@ def main():
                         "bytes": alg["op"]["bytes"], "flops": alg["op"]["flops"]},
         "stage_ms": {k: v / max(calls, 1) for k, v in stage_ms.items()},
         "clocks": clocks,
-        "e2e": {"value": tokens / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_s * 1e3, "api": "vda_forward_host (pinned host buffers)"},
+        "e2e": None if e2e is None else {
+            "value": tokens / e2e["e2e_s"], "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
+            "d2h_bytes_per_step": e2e["d2h"], "ms_per_step": e2e["e2e_s"] * 1e3,
+            "api": "vda_forward_host (pinned host buffers)"},
         "gpu_launches": launches,
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -268,8 +268,8 @@ __device__ __forceinline__ uint32_t mimg_offset(int j, int k) {
 __global__ void __launch_bounds__(256)
 k_gj_inverse_img(const float* __restrict__ A, uint8_t* __restrict__ Mimg, float* __restrict__ M_f32) {
   constexpr int D = kD, BS = 8;
-  __shared__ float s_row[2][D];
-  __shared__ float s_col[2][D];
+  __shared__ __align__(16) float s_row[2][D];
+  __shared__ __align__(16) float s_col[2][D];
   const float* Ax = A + (size_t)blockIdx.x * kDD;
   const int tid = threadIdx.x;
   const int bi = tid >> 4, bj = tid & 15;
@@ -300,10 +300,16 @@ k_gj_inverse_img(const float* __restrict__ A, uint8_t* __restrict__ Mimg, float*
       __syncthreads();
       const float pinv = 1.0f / s_row[buf][k];
       float c[BS], rs[BS];
-#pragma unroll
-      for (int i = 0; i < BS; ++i) c[i] = s_col[buf][r0 + i];
-#pragma unroll
-      for (int j = 0; j < BS; ++j) rs[j] = s_row[buf][c0 + j] * pinv;
+      {
+        const float4 c_lo = *reinterpret_cast<const float4*>(&s_col[buf][r0]);
+        const float4 c_hi = *reinterpret_cast<const float4*>(&s_col[buf][r0 + 4]);
+        const float4 r_lo = *reinterpret_cast<const float4*>(&s_row[buf][c0]);
+        const float4 r_hi = *reinterpret_cast<const float4*>(&s_row[buf][c0 + 4]);
+        c[0] = c_lo.x; c[1] = c_lo.y; c[2] = c_lo.z; c[3] = c_lo.w;
+        c[4] = c_hi.x; c[5] = c_hi.y; c[6] = c_hi.z; c[7] = c_hi.w;
+        rs[0] = r_lo.x * pinv; rs[1] = r_lo.y * pinv; rs[2] = r_lo.z * pinv; rs[3] = r_lo.w * pinv;
+        rs[4] = r_hi.x * pinv; rs[5] = r_hi.y * pinv; rs[6] = r_hi.z * pinv; rs[7] = r_hi.w * pinv;
+      }
 #pragma unroll
       for (int i = 0; i < BS; ++i)
 #pragma unroll
@@ -542,11 +548,15 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
 //   S~ = fwd[max(0, c - w)] + rev[min(NC, c + w + 1)]   (Appendix A.3)
 // TMEM lane = token row: RMSNorm is a per-thread sum of squares.  Gates come
 // through TMA as well; outputs are stored as 16-B vectors, rows past the
-// chunk end are skipped.
-// Warps 0-3: epilogue + S~ builder; warp 4: TMA producer; warp 5: MMA issuer.
+// chunk end are skipped.  The gate is sigmoid(g) = (1 + tanh(g/2)) / 2 with
+// the hardware tanh (one XU instruction per element), and the factor 1/2 is
+// folded into the RMSNorm weight held in shared memory.
+// Warps 0-3: epilogue + S~ builder; warp 4: Q producer; warp 5: MMA issuer;
+// warp 6: gate producer (separate producers keep Q loads running ahead of
+// the epilogue's release of gate stages).
 // ===========================================================================
 struct ReadoutCfg {
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 224;
   static constexpr int TILE = 128;
   static constexpr uint32_t TILE_BYTES = TILE * 256;           // 128 rows x 128 bf16
   static constexpr uint32_t OFF_S = 0;                         // S~ hi (32 KB) + lo (32 KB)
@@ -612,7 +622,7 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (tid < kD) sw[tid] = w[tid];
+  if (tid < kD) sw[tid] = 0.5f * w[tid];
   if (warp == 5) {
     tmem_alloc(smem_u32(tmem_slot), 256);
     tmem_relinquish();
@@ -624,27 +634,26 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
   const long long tokens_per_head = (long long)g.T * g.U;
   int last_q[2] = {-1, -1}, last_g[2] = {-1, -1};   // producer: last tile issued per stage
 
-  if (warp == 4) {
-    // ---------------- TMA producer: Q and gate tiles
+  if (warp == 4 || warp == 6) {
+    // ---------------- TMA producers: Q tiles (warp 4), gate tiles (warp 6)
     if (lane == 0) {
+      const bool is_q = warp == 4;
+      const int FULLB = is_q ? QFULL : GFULL, EMPTYB = is_q ? QEMPTY : GEMPTY;
+      const CUtensorMap* map = is_q ? &tmQ : &tmG;
+      const uint32_t base = sbase + (is_q ? C::OFF_Q : C::OFF_G);
+      int* last = is_q ? last_q : last_g;
       int k = 0;
       for (long long gt = t_begin; gt < t_end; ++gt, ++k) {
         int bh, c, tr, rows;
         tile_coords(g, gt, bh, c, tr, rows);
         const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.chunk * g.U + tr);
         const uint32_t s = (uint32_t)k & 1u, ph = ((uint32_t)k >> 1) & 1u;
-        if (!mbar_wait(BAR(QEMPTY + s), ph ^ 1u, abort_flag)) break;
-        mbar_arrive_expect_tx(BAR(QFULL + s), C::TILE_BYTES);
-        const uint32_t qd = sbase + C::OFF_Q + s * C::TILE_BYTES;
-        tma_load_2d(qd, &tmQ, 0, row0, BAR(QFULL + s));
-        tma_load_2d(qd + C::TILE_BYTES / 2, &tmQ, 64, row0, BAR(QFULL + s));
-        last_q[s] = k;
-        if (!mbar_wait(BAR(GEMPTY + s), ph ^ 1u, abort_flag)) break;
-        mbar_arrive_expect_tx(BAR(GFULL + s), C::TILE_BYTES);
-        const uint32_t gd = sbase + C::OFF_G + s * C::TILE_BYTES;
-        tma_load_2d(gd, &tmG, 0, row0, BAR(GFULL + s));
-        tma_load_2d(gd + C::TILE_BYTES / 2, &tmG, 64, row0, BAR(GFULL + s));
-        last_g[s] = k;
+        if (!mbar_wait(BAR(EMPTYB + s), ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(BAR(FULLB + s), C::TILE_BYTES);
+        const uint32_t dst = base + s * C::TILE_BYTES;
+        tma_load_2d(dst, map, 0, row0, BAR(FULLB + s));
+        tma_load_2d(dst + C::TILE_BYTES / 2, map, 64, row0, BAR(FULLB + s));
+        last[s] = k;
       }
     }
   } else if (warp == 5) {
@@ -730,13 +739,20 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       tc_fence_after();
       float o[kD];
       const uint32_t trow = trow_base + s * 128u;
-#pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        uint32_t v[32];
-        tmem_ld32(trow + cb * 32, v);
+      {
+        uint32_t v0[32], v1[32], v2[32], v3[32];
+        tmem_ld32(trow, v0);
+        tmem_ld32(trow + 32, v1);
+        tmem_ld32(trow + 64, v2);
+        tmem_ld32(trow + 96, v3);
         tmem_wait_ld();
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) o[cb * 32 + c2] = __uint_as_float(v[c2]);
+        for (int c2 = 0; c2 < 32; ++c2) {
+          o[c2] = __uint_as_float(v0[c2]);
+          o[32 + c2] = __uint_as_float(v1[c2]);
+          o[64 + c2] = __uint_as_float(v2[c2]);
+          o[96 + c2] = __uint_as_float(v3[c2]);
+        }
       }
       tc_fence_before();
       mbar_arrive(BAR(TEMPTY + s));
@@ -752,14 +768,19 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       for (int cc = 0; cc < 16; ++cc) {
         const uint32_t off = (uint32_t)(cc >> 3) * (C::TILE_BYTES / 2) + sw128_offset((uint32_t)r, (uint32_t)((cc & 7) * 8));
         const uint4 gv = *reinterpret_cast<const uint4*>(gt_s + off);
+        const float4 wa = *reinterpret_cast<const float4*>(sw + cc * 8);
+        const float4 wb = *reinterpret_cast<const float4*>(sw + cc * 8 + 4);
+        const float wh[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
         const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
         uint32_t yw[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int i0 = cc * 8 + 2 * q;
           const float g0 = __uint_as_float(gw[q] << 16), g1 = __uint_as_float(gw[q] & 0xFFFF0000u);
-          const float y0 = o[i0] * rinv * sw[i0] / (1.0f + __expf(-g0));
-          const float y1 = o[i0 + 1] * rinv * sw[i0 + 1] / (1.0f + __expf(-g1));
+          // y = w * o * rinv * sigmoid(g),  sigmoid(g) = (1 + tanh(g / 2)) / 2, w/2 in wh
+          const float a0 = o[i0] * rinv * wh[2 * q], a1 = o[i0 + 1] * rinv * wh[2 * q + 1];
+          const float y0 = fmaf(a0, tanh_approx(0.5f * g0), a0);
+          const float y1 = fmaf(a1, tanh_approx(0.5f * g1), a1);
           yw[q] = pack_bf16(y0, y1);
         }
         if (valid) *reinterpret_cast<uint4*>(orow + cc * 8) = make_uint4(yw[0], yw[1], yw[2], yw[3]);
@@ -774,11 +795,11 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
-  if (warp == 4 && lane == 0 && *abort_flag) {  // let issued copies land before the CTA exits
-    for (int s = 0; s < 2; ++s) {
-      if (last_q[s] >= 0) mbar_wait_drain(BAR(QFULL + s), ((uint32_t)last_q[s] >> 1) & 1u);
-      if (last_g[s] >= 0) mbar_wait_drain(BAR(GFULL + s), ((uint32_t)last_g[s] >> 1) & 1u);
-    }
+  if ((warp == 4 || warp == 6) && lane == 0 && *abort_flag) {  // let issued copies land before exit
+    const int* last = warp == 4 ? last_q : last_g;
+    const int FULLB = warp == 4 ? QFULL : GFULL;
+    for (int s = 0; s < 2; ++s)
+      if (last[s] >= 0) mbar_wait_drain(BAR(FULLB + s), ((uint32_t)last[s] >> 1) & 1u);
   }
 }
 

@@ -183,6 +183,14 @@ __host__ __device__ constexpr uint32_t sw128_offset(uint32_t row, uint32_t col) 
   return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + ((col & 7u) << 1);
 }
 
+// ---------------------------------------------------------------- math
+// Hardware tanh approximation (one XU instruction; max relative error ~2^-11).
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------- bf16 helpers
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
