@@ -3,8 +3,9 @@
 //
 // Paper: "Video DeltaNet" (arXiv 2609.20744).
 //   k_stats_tc    Eq. 3b: A_t = K^T Diag(beta) K, B_t = V^T Diag(beta) K
-//   k_gj_inverse  Eq. 5 / Appendix A.1: M_t = (I + A_t)^{-1}, written as the
-//                 bf16 hi/lo operand image the scan feeds to the tensor cores
+//   k_sweep_inverse_img  Eq. 5 / Appendix A.1: M_t = (I + A_t)^{-1} by the
+//                 symmetric sweep, written as the bf16 hi/lo operand image the
+//                 scan feeds to the tensor cores
 //   k_scan_tc     Section 2.2 + Eq. 5: S_t = (S_{t-1} + B_t) M_t, both
 //                 directions, fp32 state, 3-product bf16 hi/lo split MMAs
 //   k_readout_tc  Appendix A.3 (Eq. A.4) gather, Eq. 1a readout o = S~ q,
@@ -38,10 +39,10 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 // ===========================================================================
 // k_stats_tc: per frame-head, with tokens on the MMA's K dimension,
-//   D[128 x 256] = (beta K)_hi^T [K | V]  +  [0 | (beta K)_lo^T V]
-// so D[:, 0:128] = A (bf16 beta*K) and D[:, 128:256] = B^T (beta*K split
-// into bf16 hi + lo: the B part carries ~16 significant bits, which the
-// correlated-key workload needs).  Both operands are MN-major: a TMA box of
+//   D[128 x 256] = (beta K)_hi^T [K | V]  +  (beta K)_lo^T [K | V]
+// so D[:, 0:128] = A and D[:, 128:256] = B^T with beta*K split into bf16
+// hi + lo: ~16 significant bits, which the correlated-key workload needs in
+// B, and which keeps A symmetric to ~2^-16 for the symmetric-sweep inverse.  Both operands are MN-major: a TMA box of
 // 64 channels x 64 tokens lands as 64 rows of 128 B with the 128-B swizzle.
 //
 // Persistent CTAs (one per SM) walk frame-heads fh = blockIdx.x + i*grid.
@@ -130,7 +131,6 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
     // ---------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdN256 = idesc_bf16(128, 256, 1, 1);
-      constexpr uint32_t kIdN128 = idesc_bf16(128, 128, 1, 1);
       uint32_t it = 0, lf = 0;
       bool ok = true;
       for (int fh = blockIdx.x; ok && fh < FH; fh += gridDim.x, ++lf) {
@@ -148,8 +148,8 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
             const uint32_t ko = (uint32_t)ks * 2048u;
             mma_bf16_ss(d, desc_sw128(st + C::OFF_H + ko, C::BLK, 1024),
                         desc_sw128(st + C::OFF_KV + ko, C::BLK, 1024), kIdN256, (tile | ks) != 0);
-            mma_bf16_ss(d + 128u, desc_sw128(st + C::OFF_L + ko, C::BLK, 1024),
-                        desc_sw128(st + C::OFF_KV + 2 * C::BLK + ko, C::BLK, 1024), kIdN128, 1u);
+            mma_bf16_ss(d, desc_sw128(st + C::OFF_L + ko, C::BLK, 1024),
+                        desc_sw128(st + C::OFF_KV + ko, C::BLK, 1024), kIdN256, 1u);
           }
           mma_commit(BAR(EMPTY + s));
         }
@@ -253,102 +253,139 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
 }
 
 // ===========================================================================
-// Gauss-Jordan inverse (same elimination as k_gj_inverse in kernels_simt.cuh)
-// writing M = (I + A)^{-1} as the scan's tensor-core A operand: for the
-// product S_new[n][j] = sum_k X[n][k] M[k][j] the MMA computes
-// D[j][n] = sum_k M[k][j] X[n][k], i.e. operand element (j, k) = M[k][j],
-// MN-major (j contiguous) with the 128-B swizzle: two 64-column blocks of
-// 128 k-rows x 128 B.  M is stored split into bf16 hi (bytes [0, 32K)) and lo
-// (bytes [32K, 64K)); optionally M is also written as fp32 (debug output).
+// k_sweep_inverse_img: M = (I + A)^{-1} with the symmetric sweep operator.
+// I + A is symmetric positive definite, so sweeping every pivot k in turn,
+//   p = a_kk,  c = column k,
+//   a_ij <- a_ij - c_i c_j / p   (i, j != k)
+//   a_ik = a_ki <- c_i / p       (i != k)
+//   a_kk <- -1 / p
+// keeps the matrix symmetric and ends at -(I + A)^{-1}; every pivot is >= 1,
+// so no pivoting is needed.  Only the lower-triangle 8 x 8 blocks are kept
+// (136 threads, one block each in registers: half the FMAs of a full
+// Gauss-Jordan sweep), and the pivot row is the pivot column, so one vector
+// of 128 values per step is published through shared memory (16 threads
+// write 8 values each; double-buffered, one barrier per step).
+// Output: the scan's operand image, element (j, k) = M[k][j], MN-major,
+// 128-B swizzle, bf16 hi at [0, 32K) and lo at [32K, 64K) per frame-head,
+// written from each block and from its mirror; optional fp32 copy of M.
 // ===========================================================================
 __device__ __forceinline__ uint32_t mimg_offset(int j, int k) {
   return (uint32_t)(j >> 6) * 16384u + sw128_offset((uint32_t)k, (uint32_t)(j & 63));
 }
 
-__global__ void __launch_bounds__(256)
-k_gj_inverse_img(const float* __restrict__ A, uint8_t* __restrict__ Mimg, float* __restrict__ M_f32) {
+__device__ __forceinline__ void store_img_chunk(uint8_t* img, uint32_t off, const float (&x)[8]) {
+  uint32_t hw[4], lw[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float h0, l0, h1, l1;
+    split_bf16(x[2 * q], h0, l0);
+    split_bf16(x[2 * q + 1], h1, l1);
+    hw[q] = pack_bf16(h0, h1);
+    lw[q] = pack_bf16(l0, l1);
+  }
+  *reinterpret_cast<uint4*>(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  *reinterpret_cast<uint4*>(img + kImgHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+}
+
+constexpr int kSweepThreads = 160;   // 136 lower-triangle blocks + 24 idle lanes
+
+__global__ void __launch_bounds__(kSweepThreads, 3)
+k_sweep_inverse_img(const float* __restrict__ A, uint8_t* __restrict__ Mimg, float* __restrict__ M_f32) {
   constexpr int D = kD, BS = 8;
-  __shared__ __align__(16) float s_row[2][D];
-  __shared__ __align__(16) float s_col[2][D];
-  const float* Ax = A + (size_t)blockIdx.x * kDD;
-  const int tid = threadIdx.x;
-  const int bi = tid >> 4, bj = tid & 15;
+  __shared__ __align__(16) float s_c[2][D];
+  const int t = threadIdx.x;
+  const bool active = t < 136;
+  int bi = 0;
+  while ((bi + 1) * (bi + 2) / 2 <= t && bi < 15) ++bi;
+  const int bj = active ? t - bi * (bi + 1) / 2 : 0;
+  if (!active) bi = 0;
   const int r0 = bi * BS, c0 = bj * BS;
+  const float* Ax = A + (size_t)blockIdx.x * kDD;
+
   float a[BS][BS];
 #pragma unroll
   for (int i = 0; i < BS; ++i) {
-    const float4 x0 = *reinterpret_cast<const float4*>(Ax + (size_t)(r0 + i) * D + c0);
-    const float4 x1 = *reinterpret_cast<const float4*>(Ax + (size_t)(r0 + i) * D + c0 + 4);
+    float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
+    if (active) {
+      x0 = *reinterpret_cast<const float4*>(Ax + (size_t)(r0 + i) * D + c0);
+      x1 = *reinterpret_cast<const float4*>(Ax + (size_t)(r0 + i) * D + c0 + 4);
+    }
     a[i][0] = x0.x; a[i][1] = x0.y; a[i][2] = x0.z; a[i][3] = x0.w;
     a[i][4] = x1.x; a[i][5] = x1.y; a[i][6] = x1.z; a[i][7] = x1.w;
-#pragma unroll
-    for (int j = 0; j < BS; ++j) a[i][j] += ((r0 + i) == (c0 + j)) ? 1.f : 0.f;
+    if (active && bi == bj) a[i][i] += 1.f;
   }
+
   for (int kb = 0; kb < 16; ++kb) {
 #pragma unroll
     for (int kk = 0; kk < BS; ++kk) {
       const int k = kb * BS + kk;
-      const int buf = k & 1;
-      if (bi == kb) {
-#pragma unroll
-        for (int j = 0; j < BS; ++j) s_row[buf][c0 + j] = a[kk][j];
-      }
-      if (bj == kb) {
-#pragma unroll
-        for (int i = 0; i < BS; ++i) s_col[buf][r0 + i] = a[i][kk];
+      float* c = s_c[k & 1];
+      if (active) {
+        if (bi == kb) {          // local row kk = a_(k, c0..c0+7) = column k at rows c0..c0+7
+          *reinterpret_cast<float4*>(c + c0) = make_float4(a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
+          *reinterpret_cast<float4*>(c + c0 + 4) = make_float4(a[kk][4], a[kk][5], a[kk][6], a[kk][7]);
+        } else if (bj == kb) {   // local column kk = a_(r0..r0+7, k)
+          *reinterpret_cast<float4*>(c + r0) = make_float4(a[0][kk], a[1][kk], a[2][kk], a[3][kk]);
+          *reinterpret_cast<float4*>(c + r0 + 4) = make_float4(a[4][kk], a[5][kk], a[6][kk], a[7][kk]);
+        }
       }
       __syncthreads();
-      const float pinv = 1.0f / s_row[buf][k];
-      float c[BS], rs[BS];
+      const float pinv = __frcp_rn(c[k]);
+      float fr[BS], cs[BS];
       {
-        const float4 c_lo = *reinterpret_cast<const float4*>(&s_col[buf][r0]);
-        const float4 c_hi = *reinterpret_cast<const float4*>(&s_col[buf][r0 + 4]);
-        const float4 r_lo = *reinterpret_cast<const float4*>(&s_row[buf][c0]);
-        const float4 r_hi = *reinterpret_cast<const float4*>(&s_row[buf][c0 + 4]);
-        c[0] = c_lo.x; c[1] = c_lo.y; c[2] = c_lo.z; c[3] = c_lo.w;
-        c[4] = c_hi.x; c[5] = c_hi.y; c[6] = c_hi.z; c[7] = c_hi.w;
-        rs[0] = r_lo.x * pinv; rs[1] = r_lo.y * pinv; rs[2] = r_lo.z * pinv; rs[3] = r_lo.w * pinv;
-        rs[4] = r_hi.x * pinv; rs[5] = r_hi.y * pinv; rs[6] = r_hi.z * pinv; rs[7] = r_hi.w * pinv;
+        const float4 r_lo = *reinterpret_cast<const float4*>(c + r0);
+        const float4 r_hi = *reinterpret_cast<const float4*>(c + r0 + 4);
+        const float4 s_lo = *reinterpret_cast<const float4*>(c + c0);
+        const float4 s_hi = *reinterpret_cast<const float4*>(c + c0 + 4);
+        fr[0] = r_lo.x * pinv; fr[1] = r_lo.y * pinv; fr[2] = r_lo.z * pinv; fr[3] = r_lo.w * pinv;
+        fr[4] = r_hi.x * pinv; fr[5] = r_hi.y * pinv; fr[6] = r_hi.z * pinv; fr[7] = r_hi.w * pinv;
+        cs[0] = s_lo.x; cs[1] = s_lo.y; cs[2] = s_lo.z; cs[3] = s_lo.w;
+        cs[4] = s_hi.x; cs[5] = s_hi.y; cs[6] = s_hi.z; cs[7] = s_hi.w;
       }
 #pragma unroll
       for (int i = 0; i < BS; ++i)
 #pragma unroll
-        for (int j = 0; j < BS; ++j) a[i][j] = fmaf(-c[i], rs[j], a[i][j]);
+        for (int j = 0; j < BS; ++j) a[i][j] = fmaf(-fr[i], cs[j], a[i][j]);
       if (bi == kb) {
 #pragma unroll
-        for (int j = 0; j < BS; ++j) a[kk][j] = rs[j];
+        for (int j = 0; j < BS; ++j) a[kk][j] = cs[j] * pinv;
       }
       if (bj == kb) {
 #pragma unroll
-        for (int i = 0; i < BS; ++i) a[i][kk] = -c[i] * pinv;
+        for (int i = 0; i < BS; ++i) a[i][kk] = fr[i];
       }
-      if (bi == kb && bj == kb) a[kk][kk] = pinv;
+      if (bi == kb && bj == kb) a[kk][kk] = -pinv;
     }
   }
-  // a[i][j] = M[r0 + i][c0 + j]: row index = k, column index = j of the operand
+  if (!active) return;
+
+  // a = -M on this block; write the block (rows r0.., columns c0..) and its mirror
   uint8_t* img = Mimg + (size_t)blockIdx.x * kImgBytes;
 #pragma unroll
   for (int i = 0; i < BS; ++i) {
-    uint32_t hw[4], lw[4];
+    float x[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float h0, l0, h1, l1;
-      split_bf16(a[i][2 * q], h0, l0);
-      split_bf16(a[i][2 * q + 1], h1, l1);
-      hw[q] = pack_bf16(h0, h1);
-      lw[q] = pack_bf16(l0, l1);
+    for (int j = 0; j < BS; ++j) x[j] = -a[i][j];
+    store_img_chunk(img, mimg_offset(c0, r0 + i), x);      // image row r0+i, columns c0..c0+7
+  }
+  if (bi != bj) {
+#pragma unroll
+    for (int j = 0; j < BS; ++j) {
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < BS; ++i) x[i] = -a[i][j];
+      store_img_chunk(img, mimg_offset(r0, c0 + j), x);    // image row c0+j, columns r0..r0+7
     }
-    const uint32_t off = mimg_offset(c0, r0 + i);   // 8 consecutive j = one 16-B chunk
-    *reinterpret_cast<uint4*>(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-    *reinterpret_cast<uint4*>(img + kImgHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
   }
   if (M_f32) {
     float* Mf = M_f32 + (size_t)blockIdx.x * kDD;
 #pragma unroll
-    for (int i = 0; i < BS; ++i) {
-      *reinterpret_cast<float4*>(Mf + (size_t)(r0 + i) * D + c0) = make_float4(a[i][0], a[i][1], a[i][2], a[i][3]);
-      *reinterpret_cast<float4*>(Mf + (size_t)(r0 + i) * D + c0 + 4) = make_float4(a[i][4], a[i][5], a[i][6], a[i][7]);
-    }
+    for (int i = 0; i < BS; ++i)
+#pragma unroll
+      for (int j = 0; j < BS; ++j) {
+        Mf[(size_t)(r0 + i) * D + c0 + j] = -a[i][j];
+        Mf[(size_t)(c0 + j) * D + r0 + i] = -a[i][j];
+      }
   }
 }
 
@@ -806,6 +843,46 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 // ===========================================================================
 // host side
 // ===========================================================================
+}  // namespace tc
+
+// With VDA_DEBUG_SYNC=1 in the environment, every stage is followed by a
+// stream synchronisation and a check of the device error word, and a failing
+// stage is named on stderr (a debugging aid; off by default).
+inline bool debug_sync_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("VDA_DEBUG_SYNC");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+inline int debug_check(const char* stage, cudaStream_t s) {
+  if (!debug_sync_enabled()) return VDA_OK;
+  const cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "vda: stage %s failed: %s\n", stage, cudaGetErrorString(e));
+    return VDA_ERR_CUDA;
+  }
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) == cudaSuccess && word != 0) {
+    fprintf(stderr, "vda: stage %s gave up a bounded wait (device error word %u)\n", stage, word);
+    return VDA_ERR_TIMEOUT;
+  }
+  return VDA_OK;
+}
+
+// Status of the launch just made; names the kernel and the CUDA error on
+// stderr in debug mode.
+inline int launch_status(const char* kernel) {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return VDA_OK;
+  if (debug_sync_enabled()) fprintf(stderr, "vda: launch of %s failed: %s\n", kernel, cudaGetErrorString(e));
+  return VDA_ERR_CUDA;
+}
+
+namespace tc {
+
 inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -861,12 +938,12 @@ inline int launch_stats(const void* K, const void* V, const float* beta, int U, 
     return VDA_ERR_CUDA;
   const int grid = (int)std::min<size_t>(FH, (size_t)num_sms());
   k_stats_tc<<<grid, StatsCfg::THREADS, StatsCfg::SMEM, s>>>(tmK, tmV, beta, U, (int)FH, A, B);
-  return cudaGetLastError() == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+  return launch_status("k_stats_tc");
 }
 
 inline int launch_inverse_img(const float* A, uint8_t* Mimg, float* M_f32, size_t FH, cudaStream_t s) {
-  k_gj_inverse_img<<<(unsigned)FH, 256, 0, s>>>(A, Mimg, M_f32);
-  return cudaGetLastError() == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+  k_sweep_inverse_img<<<(unsigned)FH, kSweepThreads, 0, s>>>(A, Mimg, M_f32);
+  return launch_status("k_sweep_inverse_img");
 }
 
 inline int launch_scan(const uint8_t* Mimg, const float* Bm, const float* S0f, const float* S0r, float* states,
@@ -876,7 +953,7 @@ inline int launch_scan(const uint8_t* Mimg, const float* Bm, const float* S0f, c
     return VDA_ERR_CUDA;
   dim3 grid((unsigned)BH, (unsigned)ndir);
   k_scan_tc<<<grid, ScanCfg::THREADS, ScanCfg::SMEM, s>>>(Mimg, Bm, S0f, S0r, states, (int)BH, T, chunk, NC);
-  return cudaGetLastError() == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+  return launch_status("k_scan_tc");
 }
 
 inline int launch_readout(const void* Q, const void* G, const float* w, const float* states, void* out,
@@ -899,7 +976,7 @@ inline int launch_readout(const void* Q, const void* G, const float* w, const fl
   const int grid = (int)std::min<long long>(g.total, (long long)num_sms());
   k_readout_tc<<<grid, ReadoutCfg::THREADS, ReadoutCfg::SMEM, s>>>(
       tmQ, tmG, w, states, static_cast<__nv_bfloat16*>(out), g, eps);
-  return cudaGetLastError() == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+  return launch_status("k_readout_tc");
 }
 
 }  // namespace tc
@@ -915,33 +992,6 @@ inline size_t tc_extra_workspace_bytes(bool tc, size_t FH, int d) {
 }
 
 inline int tc_launches_per_forward() { return 4; }
-
-// With VDA_DEBUG_SYNC=1 in the environment, every stage is followed by a
-// stream synchronisation and a check of the device error word, and a failing
-// stage is named on stderr (a debugging aid; off by default).
-inline bool debug_sync_enabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("VDA_DEBUG_SYNC");
-    v = (e && e[0] == '1') ? 1 : 0;
-  }
-  return v == 1;
-}
-
-inline int debug_check(const char* stage, cudaStream_t s) {
-  if (!debug_sync_enabled()) return VDA_OK;
-  const cudaError_t e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) {
-    fprintf(stderr, "vda: stage %s failed: %s\n", stage, cudaGetErrorString(e));
-    return VDA_ERR_CUDA;
-  }
-  unsigned int word = 0;
-  if (cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)) == cudaSuccess && word != 0) {
-    fprintf(stderr, "vda: stage %s gave up a bounded wait (device error word %u)\n", stage, word);
-    return VDA_ERR_TIMEOUT;
-  }
-  return VDA_OK;
-}
 
 template <typename MarkFn>
 int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_args& a, char* ws_AM,
