@@ -3,9 +3,9 @@
 //
 // Paper: "Video DeltaNet" (arXiv 2609.20744).
 //   k_stats_tc    Eq. 3b: A_t = K^T Diag(beta) K, B_t = V^T Diag(beta) K
-//   k_sweep_inverse_img  Eq. 5 / Appendix A.1: M_t = (I + A_t)^{-1} by the
-//                 symmetric sweep, written as the bf16 hi/lo operand image the
-//                 scan feeds to the tensor cores
+//   k_inverse_tc  Eq. 5 / Appendix A.1: M_t = (I + A_t)^{-1} by a block sweep
+//                 on the tensor cores, written as the bf16 hi/lo operand image
+//                 the scan feeds to the tensor cores
 //   k_scan_tc     Section 2.2 + Eq. 5: S_t = (S_{t-1} + B_t) M_t, both
 //                 directions, fp32 state, 3-product bf16 hi/lo split MMAs
 //   k_readout_tc  Appendix A.3 (Eq. A.4) gather, Eq. 1a readout o = S~ q,
@@ -46,8 +46,10 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // 64 channels x 64 tokens lands as 64 rows of 128 B with the 128-B swizzle.
 //
 // Persistent CTAs (one per SM) walk frame-heads fh = blockIdx.x + i*grid.
-// Warps: 0-3 epilogue (TMEM -> global), 4-7 scale (beta*K hi/lo),
-//        8 TMA producer, 9 MMA issuer + TMEM owner.
+// Warps: 0-3 epilogue (TMEM -> A and B, fp32, standard layouts, coalesced),
+//        4-7 scale (beta*K hi/lo), 8 TMA producer, 9 MMA issuer + TMEM
+//        owner.  Two TMEM accumulators: the epilogue of one frame-head
+//        overlaps the MMAs of the next.
 // Stage s holds K0 K1 V0 V1 (TMA), H0 H1 (hi), L0 L1 (lo): 8 x 8 KB.
 // TMEM: two 256-column accumulators (512 columns), so the epilogue of one
 // frame-head overlaps the MMAs of the next.
@@ -66,10 +68,53 @@ struct StatsCfg {
   static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
 };
 
+// byte offset of element (r, k), k < 16, in a K-major no-swizzle image
+__device__ __forceinline__ uint32_t kimg16(uint32_t r, uint32_t k) {
+  return (r >> 3) * 256u + (k >> 3) * 128u + (r & 7u) * 16u + (k & 7u) * 2u;
+}
+
+// 16 fp32 values -> bf16 hi and lo rows of two no-swizzle images
+__device__ __forceinline__ void store_row16_hilo(uint32_t img_hi, uint32_t img_lo, uint32_t r, const float (&x)[16]) {
+#pragma unroll
+  for (int kc = 0; kc < 2; ++kc) {
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float h0, l0, h1, l1;
+      split_bf16(x[8 * kc + 2 * q], h0, l0);
+      split_bf16(x[8 * kc + 2 * q + 1], h1, l1);
+      hw[q] = pack_bf16(h0, h1);
+      lw[q] = pack_bf16(l0, l1);
+    }
+    const uint32_t off = kimg16(r, 8u * kc);
+    st_shared_v4(img_hi + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+    st_shared_v4(img_lo + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+  }
+}
+
+__device__ __forceinline__ uint32_t mimg_offset(int j, int k) {
+  return (uint32_t)(j >> 6) * 16384u + sw128_offset((uint32_t)k, (uint32_t)(j & 63));
+}
+
+// 8 fp32 values -> one 16-B chunk of the bf16 hi image and of the lo image
+__device__ __forceinline__ void store_img_chunk(uint8_t* img, uint32_t off, const float (&x)[8]) {
+  uint32_t hw[4], lw[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float h0, l0, h1, l1;
+    split_bf16(x[2 * q], h0, l0);
+    split_bf16(x[2 * q + 1], h1, l1);
+    hw[q] = pack_bf16(h0, h1);
+    lw[q] = pack_bf16(l0, l1);
+  }
+  *reinterpret_cast<uint4*>(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  *reinterpret_cast<uint4*>(img + kImgHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+}
+
 __global__ void __launch_bounds__(StatsCfg::THREADS, 1)
 k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-           const float* __restrict__ beta, int U, int FH,
-           float* __restrict__ A_out, float* __restrict__ B_out) {
+           const float* __restrict__ beta, int U, int FH, float* __restrict__ A_out,
+           float* __restrict__ B_out) {
   using C = StatsCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -179,14 +224,12 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
       b_next = beta_at(nfh, ntile);
       const uint32_t s = it % C::NST, ph = (it / C::NST) & 1u;
       if (!mbar_wait(BAR(FULL + s), ph, abort_flag)) break;
-      uint8_t* stg = smem + s * C::STAGE;
-      const uint8_t* ksrc = stg + C::OFF_KV + hb * C::BLK + r * 128;
-      uint8_t* hdst = stg + C::OFF_H + hb * C::BLK + r * 128;
-      uint8_t* ldst = stg + C::OFF_L + hb * C::BLK + r * 128;
+      const uint32_t rowb = sbase + s * C::STAGE + hb * C::BLK + (uint32_t)r * 128u;
+      const uint32_t ksrc = rowb + C::OFF_KV, hdst = rowb + C::OFF_H, ldst = rowb + C::OFF_L;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const int p = (c + r) & 7;   // rotate chunks across rows: conflict-free
-        const uint4 kv = *reinterpret_cast<const uint4*>(ksrc + p * 16);
+        const uint32_t p = (uint32_t)((c + r) & 7) * 16u;   // rotate chunks across rows: conflict-free
+        const uint4 kv = ld_shared_v4(ksrc + p);
         const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
         uint32_t hw[4], lw[4];
 #pragma unroll
@@ -199,8 +242,8 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
           hw[q] = pack_bf16(h0, h1);
           lw[q] = pack_bf16(l0, l1);
         }
-        *reinterpret_cast<uint4*>(hdst + p * 16) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(ldst + p * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        st_shared_v4(hdst + p, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+        st_shared_v4(ldst + p, make_uint4(lw[0], lw[1], lw[2], lw[3]));
       }
       fence_proxy_async_smem();
       mbar_arrive(BAR(SCALED + s));
@@ -209,28 +252,29 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
       tile = ntile;
     }
   } else {
-    // ---------------- epilogue: TMEM lane i = channel i of D
+    // ---------------- epilogue: TMEM lane i = row i of D; column c of D goes to
+    // A[c][i] (A is symmetric) or B[c - 128][i]: 32 lanes store 128 contiguous bytes
     const int i = warp * 32 + lane;
+    const uint32_t lb = (uint32_t)(warp * 32) << 16;
     uint32_t lf = 0;
     for (int fh = blockIdx.x; fh < FH; fh += gridDim.x, ++lf) {
       const uint32_t buf = lf & 1u, bph = (lf >> 1) & 1u;
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(TFULL + buf), bph, abort_flag))) break;
       tc_fence_after();
-      const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16) + buf * 256u;
+      const uint32_t tA = tmem + buf * 256u;
       float* Af = A_out + (size_t)fh * kDD;
       float* Bf = B_out + (size_t)fh * kDD;
 #pragma unroll 1
-      for (int rr = 0; rr < 4; ++rr) {
+      for (int q = 0; q < 4; ++q) {
         uint32_t v0[32], v1[32];
-        tmem_ld32(trow + rr * 64, v0);
-        tmem_ld32(trow + rr * 64 + 32, v1);
+        tmem_ld32(lb + tA + 64u * q, v0);
+        tmem_ld32(lb + tA + 64u * q + 32u, v1);
         tmem_wait_ld();
-        if (rr == 3) {
+        if (q == 3) {
           tc_fence_before();
           mbar_arrive(BAR(TEMPTY + buf));
         }
-        // D[i][col] -> A_out[col][i] (A is symmetric) / B_out[col - 128][i]
-        float* dst = rr < 2 ? Af + (size_t)(rr * 64) * kD : Bf + (size_t)((rr - 2) * 64) * kD;
+        float* dst = q < 2 ? Af + (size_t)(64 * q) * kD : Bf + (size_t)(64 * (q - 2)) * kD;
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           dst[(size_t)c * kD + i] = __uint_as_float(v0[c]);
@@ -253,139 +297,267 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
 }
 
 // ===========================================================================
-// k_sweep_inverse_img: M = (I + A)^{-1} with the symmetric sweep operator.
-// I + A is symmetric positive definite, so sweeping every pivot k in turn,
-//   p = a_kk,  c = column k,
-//   a_ij <- a_ij - c_i c_j / p   (i, j != k)
-//   a_ik = a_ki <- c_i / p       (i != k)
-//   a_kk <- -1 / p
-// keeps the matrix symmetric and ends at -(I + A)^{-1}; every pivot is >= 1,
-// so no pivoting is needed.  Only the lower-triangle 8 x 8 blocks are kept
-// (136 threads, one block each in registers: half the FMAs of a full
-// Gauss-Jordan sweep), and the pivot row is the pivot column, so one vector
-// of 128 values per step is published through shared memory (16 threads
-// write 8 values each; double-buffered, one barrier per step).
-// Output: the scan's operand image, element (j, k) = M[k][j], MN-major,
-// 128-B swizzle, bf16 hi at [0, 32K) and lo at [32K, 64K) per frame-head,
-// written from each block and from its mirror; optional fp32 copy of M.
+// k_inverse_tc: M = (I + A)^{-1} for every frame-head, by a block sweep of the
+// symmetric positive definite I + A held in TMEM, with the rank-16 updates
+// on the tensor cores.  Sweeping every index of a symmetric matrix ends at
+// its negative inverse; with pivot blocks P = [16K, 16K + 16), one block step
+//   G = -P^{-1}                 (16 x 16 sweep with warp shuffles)
+//   A_ij += (C G)_i C_j^T       (i, j outside P; C = A[:, P]; one MMA)
+//   A_iP = W_i = -(C G)_i,  A_PP = G,  A_Pj = W_j^T   (fix-ups)
+// sweeps the 16 indices of P at once.  Every pivot block of an SPD matrix's
+// Schur complement is SPD, so no pivoting is needed.  C, G and C G go to the
+// tensor cores as bf16 hi + lo (three products, ~16 significant bits).
+// Three warpgroups per CTA work on three matrices at once (own TMEM
+// columns, shared-memory workspace, named barrier and completion barrier),
+// so their round trips to the tensor pipe interleave.  In: A rows (fp32, from
+// k_stats_tc).  Out: the scan's M operand image (element (j, k) = M[k][j],
+// MN-major, 128-B swizzle, bf16 hi / lo halves) and optionally M in fp32.
 // ===========================================================================
-__device__ __forceinline__ uint32_t mimg_offset(int j, int k) {
-  return (uint32_t)(j >> 6) * 16384u + sw128_offset((uint32_t)k, (uint32_t)(j & 63));
-}
+struct InvCfg {
+  static constexpr int GROUPS = 3;
+  static constexpr int THREADS = 128 * GROUPS;
+  static constexpr uint32_t TCOLS = 160;     // TMEM columns per group: A (128) + C G scratch (16)
+  static constexpr uint32_t SW_BYTES = 25728; // per-group workspace (see SW_* below)
+  static constexpr uint32_t BAR_OFF = GROUPS * SW_BYTES;
+  static constexpr size_t SMEM = BAR_OFF + GROUPS * 8 + 16 + 1024;
+};
+// per-group workspace: K-major no-swizzle operand images (rows of 16 bf16)
+constexpr uint32_t SW_CH = 0, SW_CL = 4096;        // panel C, 128 rows
+constexpr uint32_t SW_GH = 8192, SW_GL = 8704;     // G = -P^{-1}, 16 rows
+constexpr uint32_t SW_CGH = 9216, SW_CGL = 13312;  // C G, 128 rows
+constexpr uint32_t SW_W = 17408;                   // W^T = (-C G)^T, fp32 [16][128]
+constexpr uint32_t SW_PB = 25600;                  // pivot-row broadcast, fp32 [2][16]
 
-__device__ __forceinline__ void store_img_chunk(uint8_t* img, uint32_t off, const float (&x)[8]) {
-  uint32_t hw[4], lw[4];
+// One warpgroup sweeps the matrix in TMEM columns [tA, tA + 128); thread i =
+// TMEM lane i; gw = warp index within the group.  Returns false on abort.
+__device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t tW, uint32_t lb, uint32_t swb,
+                                                   uint32_t bid, uint32_t sbar, uint32_t& sweep_phase,
+                                                   volatile int* abort_flag, int i, int gw, int lane) {
+  constexpr uint32_t kId16 = idesc_bf16(128, 16, 0, 0);
+  constexpr uint32_t kId128 = idesc_bf16(128, 128, 0, 0);
+  bool ok = true;
+  // block sweep of I + A, pivot blocks P = [16K, 16K + 16):
+  //   G = -P^{-1} (16 x 16 sweep in the half-warp owning the rows of P),
+  //   C = A[:, P], A += (C G) C^T on the tensor cores (3-product bf16
+  //   split, into A's own TMEM columns), then the pivot columns become
+  //   W = -C G (G on the pivot rows) and the pivot rows W^T.  After all
+  //   eight blocks TMEM holds -(I + A)^{-1}.
+#pragma unroll 1
+  for (int K = 0; K < 8; ++K) {
+    const uint32_t p0 = 16u * (uint32_t)K;
+    const bool inP = (i >> 4) == K;
+    const bool pwarp = gw == (K >> 1);
+    float c[16];
+    {
+      uint32_t v[16];
+      tmem_ld16(lb + tA + p0, v);
+      tmem_wait_ld();
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    float h0, l0, h1, l1;
-    split_bf16(x[2 * q], h0, l0);
-    split_bf16(x[2 * q + 1], h1, l1);
-    hw[q] = pack_bf16(h0, h1);
-    lw[q] = pack_bf16(l0, l1);
-  }
-  *reinterpret_cast<uint4*>(img + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-  *reinterpret_cast<uint4*>(img + kImgHalf + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-}
-
-constexpr int kSweepThreads = 160;   // 136 lower-triangle blocks + 24 idle lanes
-
-__global__ void __launch_bounds__(kSweepThreads, 3)
-k_sweep_inverse_img(const float* __restrict__ A, uint8_t* __restrict__ Mimg, float* __restrict__ M_f32) {
-  constexpr int D = kD, BS = 8;
-  __shared__ __align__(16) float s_c[2][D];
-  const int t = threadIdx.x;
-  const bool active = t < 136;
-  int bi = 0;
-  while ((bi + 1) * (bi + 2) / 2 <= t && bi < 15) ++bi;
-  const int bj = active ? t - bi * (bi + 1) / 2 : 0;
-  if (!active) bi = 0;
-  const int r0 = bi * BS, c0 = bj * BS;
-  const float* Ax = A + (size_t)blockIdx.x * kDD;
-
-  float a[BS][BS];
-#pragma unroll
-  for (int i = 0; i < BS; ++i) {
-    float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
-    if (active) {
-      x0 = *reinterpret_cast<const float4*>(Ax + (size_t)(r0 + i) * D + c0);
-      x1 = *reinterpret_cast<const float4*>(Ax + (size_t)(r0 + i) * D + c0 + 4);
+      for (int t = 0; t < 16; ++t)
+        c[t] = __uint_as_float(v[t]) + ((inP && (i & 15) == t) ? 1.f : 0.f);   // identity on P's diagonal
     }
-    a[i][0] = x0.x; a[i][1] = x0.y; a[i][2] = x0.z; a[i][3] = x0.w;
-    a[i][4] = x1.x; a[i][5] = x1.y; a[i][6] = x1.z; a[i][7] = x1.w;
-    if (active && bi == bj) a[i][i] += 1.f;
-  }
-
-  for (int kb = 0; kb < 16; ++kb) {
+    float g[16];
 #pragma unroll
-    for (int kk = 0; kk < BS; ++kk) {
-      const int k = kb * BS + kk;
-      float* c = s_c[k & 1];
-      if (active) {
-        if (bi == kb) {          // local row kk = a_(k, c0..c0+7) = column k at rows c0..c0+7
-          *reinterpret_cast<float4*>(c + c0) = make_float4(a[kk][0], a[kk][1], a[kk][2], a[kk][3]);
-          *reinterpret_cast<float4*>(c + c0 + 4) = make_float4(a[kk][4], a[kk][5], a[kk][6], a[kk][7]);
-        } else if (bj == kb) {   // local column kk = a_(r0..r0+7, k)
-          *reinterpret_cast<float4*>(c + r0) = make_float4(a[0][kk], a[1][kk], a[2][kk], a[3][kk]);
-          *reinterpret_cast<float4*>(c + r0 + 4) = make_float4(a[4][kk], a[5][kk], a[6][kk], a[7][kk]);
+    for (int t = 0; t < 16; ++t) g[t] = c[t];
+    if (pwarp) {   // 16 x 16 sweep per 16-lane segment (the segment owning P is used)
+      const int r = lane & 15;
+      const uint32_t pb = swb + SW_PB + (uint32_t)(lane >> 4) * 64u;   // this segment's broadcast row
+#pragma unroll
+      for (int sidx = 0; sidx < 16; ++sidx) {
+        // row sidx = column sidx (symmetric): its owner publishes it for the segment
+        if (r == sidx) {
+#pragma unroll
+          for (int t = 0; t < 16; t += 4)
+            st_shared_v4(pb + 4u * t, make_uint4(__float_as_uint(g[t]), __float_as_uint(g[t + 1]),
+                                                 __float_as_uint(g[t + 2]), __float_as_uint(g[t + 3])));
         }
-      }
-      __syncthreads();
-      const float pinv = __frcp_rn(c[k]);
-      float fr[BS], cs[BS];
-      {
-        const float4 r_lo = *reinterpret_cast<const float4*>(c + r0);
-        const float4 r_hi = *reinterpret_cast<const float4*>(c + r0 + 4);
-        const float4 s_lo = *reinterpret_cast<const float4*>(c + c0);
-        const float4 s_hi = *reinterpret_cast<const float4*>(c + c0 + 4);
-        fr[0] = r_lo.x * pinv; fr[1] = r_lo.y * pinv; fr[2] = r_lo.z * pinv; fr[3] = r_lo.w * pinv;
-        fr[4] = r_hi.x * pinv; fr[5] = r_hi.y * pinv; fr[6] = r_hi.z * pinv; fr[7] = r_hi.w * pinv;
-        cs[0] = s_lo.x; cs[1] = s_lo.y; cs[2] = s_lo.z; cs[3] = s_lo.w;
-        cs[4] = s_hi.x; cs[5] = s_hi.y; cs[6] = s_hi.z; cs[7] = s_hi.w;
-      }
+        __syncwarp();
+        float col[16];
 #pragma unroll
-      for (int i = 0; i < BS; ++i)
+        for (int t = 0; t < 16; t += 4) {
+          const float4 x = ld_shared_f4(pb + 4u * t);
+          col[t] = x.x; col[t + 1] = x.y; col[t + 2] = x.z; col[t + 3] = x.w;
+        }
+        __syncwarp();
+        const float pinv = rcp_approx(col[sidx]);
+        const bool me = r == sidx;
+        const float f = g[sidx] * pinv;
 #pragma unroll
-        for (int j = 0; j < BS; ++j) a[i][j] = fmaf(-fr[i], cs[j], a[i][j]);
-      if (bi == kb) {
-#pragma unroll
-        for (int j = 0; j < BS; ++j) a[kk][j] = cs[j] * pinv;
+        for (int t = 0; t < 16; ++t) g[t] = me ? col[t] * pinv : fmaf(-f, col[t], g[t]);
+        g[sidx] = me ? -pinv : f;
       }
-      if (bj == kb) {
-#pragma unroll
-        for (int i = 0; i < BS; ++i) a[i][kk] = fr[i];
-      }
-      if (bi == kb && bj == kb) a[kk][kk] = -pinv;
+      if (inP) store_row16_hilo(swb + SW_GH, swb + SW_GL, (uint32_t)r, g);
     }
+    store_row16_hilo(swb + SW_CH, swb + SW_CL, (uint32_t)i, c);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_bar_sync(bid, 128);
+    if (i == 0) {   // C G -> scratch columns [128, 144) of this buffer
+      tc_fence_after();
+      const uint64_t ch = desc_noswz(swb + SW_CH, 128, 256), cl = desc_noswz(swb + SW_CL, 128, 256);
+      const uint64_t gh = desc_noswz(swb + SW_GH, 128, 256), gl = desc_noswz(swb + SW_GL, 128, 256);
+      mma_bf16_ss(tW, ch, gh, kId16, 0u);
+      mma_bf16_ss(tW, ch, gl, kId16, 1u);
+      mma_bf16_ss(tW, cl, gh, kId16, 1u);
+      mma_commit(sbar);
+    }
+    ok = named_bar_and(bid, 128, mbar_wait(sbar, sweep_phase, abort_flag));
+    sweep_phase ^= 1u;
+    if (!ok) return false;
+    tc_fence_after();
+    float cg[16];
+    {
+      uint32_t v[16];
+      tmem_ld16(lb + tW, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int t = 0; t < 16; ++t) cg[t] = __uint_as_float(v[t]);
+    }
+    store_row16_hilo(swb + SW_CGH, swb + SW_CGL, (uint32_t)i, cg);
+#pragma unroll
+    for (int t = 0; t < 16; ++t)   // W^T[t][i] = -(C G)[i][t]; lanes write consecutive words
+      st_shared_f1(swb + SW_W + (uint32_t)t * 512u + 4u * (uint32_t)i, -cg[t]);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_bar_sync(bid, 128);
+    if (i == 0) {   // A += (C G) C^T
+      tc_fence_after();
+      const uint64_t ch = desc_noswz(swb + SW_CH, 128, 256), cl = desc_noswz(swb + SW_CL, 128, 256);
+      const uint64_t qh = desc_noswz(swb + SW_CGH, 128, 256), ql = desc_noswz(swb + SW_CGL, 128, 256);
+      mma_bf16_ss(tA, qh, ch, kId128, 1u);
+      mma_bf16_ss(tA, qh, cl, kId128, 1u);
+      mma_bf16_ss(tA, ql, ch, kId128, 1u);
+      mma_commit(sbar);
+    }
+    ok = named_bar_and(bid, 128, mbar_wait(sbar, sweep_phase, abort_flag));
+    sweep_phase ^= 1u;
+    if (!ok) return false;
+    tc_fence_after();
+    // (3) fix-ups of the pivot columns (all rows) and pivot rows
+    if (pwarp) {   // rewrite the full rows of this warp's 32 lanes
+      const int r = lane & 15;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t v[32];
+        tmem_ld32(lb + tA + 32u * q, v);
+        tmem_wait_ld();
+        if (inP) {   // pivot rows: W_j^T for the columns outside P
+#pragma unroll
+          for (int t = 0; t < 32; t += 4) {
+            const float4 x = ld_shared_f4(swb + SW_W + (uint32_t)r * 512u + 4u * (uint32_t)(32 * q + t));
+            v[t] = __float_as_uint(x.x); v[t + 1] = __float_as_uint(x.y);
+            v[t + 2] = __float_as_uint(x.z); v[t + 3] = __float_as_uint(x.w);
+          }
+        }
+        if (q == (K >> 1)) {   // the 16 pivot columns sit in this 32-column chunk
+          if ((K & 1) == 0) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) v[t] = __float_as_uint(inP ? g[t] : -cg[t]);
+          } else {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) v[16 + t] = __float_as_uint(inP ? g[t] : -cg[t]);
+          }
+        }
+        tmem_st32(lb + tA + 32u * q, v);
+      }
+    } else {
+      uint32_t v[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) v[t] = __float_as_uint(-cg[t]);
+      tmem_st16(lb + tA + p0, v);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    named_bar_sync(bid, 128);
+    tc_fence_after();
   }
-  if (!active) return;
+  return true;
+}
 
-  // a = -M on this block; write the block (rows r0.., columns c0..) and its mirror
-  uint8_t* img = Mimg + (size_t)blockIdx.x * kImgBytes;
-#pragma unroll
-  for (int i = 0; i < BS; ++i) {
-    float x[8];
-#pragma unroll
-    for (int j = 0; j < BS; ++j) x[j] = -a[i][j];
-    store_img_chunk(img, mimg_offset(c0, r0 + i), x);      // image row r0+i, columns c0..c0+7
+__global__ void __launch_bounds__(InvCfg::THREADS, 1)
+k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, float* __restrict__ M_dbg) {
+  using C = InvCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::GROUPS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = warp >> 2, gw = warp & 3;
+  const int i = gw * 32 + lane;
+  const uint32_t sbar = sbase + C::BAR_OFF + 8u * (uint32_t)g;
+  if (tid == 0) {
+    for (int q = 0; q < C::GROUPS; ++q) mbar_init(sbase + C::BAR_OFF + 8u * q, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
-  if (bi != bj) {
-#pragma unroll
-    for (int j = 0; j < BS; ++j) {
-      float x[8];
-#pragma unroll
-      for (int i = 0; i < BS; ++i) x[i] = -a[i][j];
-      store_img_chunk(img, mimg_offset(r0, c0 + j), x);    // image row c0+j, columns r0..r0+7
-    }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
   }
-  if (M_f32) {
-    float* Mf = M_f32 + (size_t)blockIdx.x * kDD;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tA = tmem + C::TCOLS * (uint32_t)g, tW = tA + 128u;
+  const uint32_t lb = (uint32_t)(gw * 32) << 16;
+  const uint32_t swb = sbase + C::SW_BYTES * (uint32_t)g;
+  const uint32_t bid = 1u + (uint32_t)g;
+  uint32_t sweep_phase = 0;
+
+  for (int m = blockIdx.x * C::GROUPS + g; m < FH; m += gridDim.x * C::GROUPS) {
+    // row i of A -> TMEM lane i
+    const float4* Ar = reinterpret_cast<const float4*>(A + (size_t)m * kDD + (size_t)i * kD);
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+      uint32_t v[32];
 #pragma unroll
-    for (int i = 0; i < BS; ++i)
-#pragma unroll
-      for (int j = 0; j < BS; ++j) {
-        Mf[(size_t)(r0 + i) * D + c0 + j] = -a[i][j];
-        Mf[(size_t)(c0 + j) * D + r0 + i] = -a[i][j];
+      for (int c = 0; c < 8; ++c) {
+        const float4 x = __ldg(Ar + 8 * q + c);
+        v[4 * c] = __float_as_uint(x.x); v[4 * c + 1] = __float_as_uint(x.y);
+        v[4 * c + 2] = __float_as_uint(x.z); v[4 * c + 3] = __float_as_uint(x.w);
       }
+      tmem_st32(lb + tA + 32u * q, v);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    named_bar_sync(bid, 128);
+    tc_fence_after();
+    if (!sweep_inverse_tmem(tA, tW, lb, swb, bid, sbar, sweep_phase, abort_flag, i, gw, lane)) break;
+    // M = -(swept matrix): row i -> operand image row i (k index), debug copy
+    uint8_t* img = Mimg + (size_t)m * kImgBytes;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+      uint32_t v[32];
+      tmem_ld32(lb + tA + 32u * q, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = -__uint_as_float(v[8 * cc + e]);
+        store_img_chunk(img, mimg_offset(32 * q + 8 * cc, i), x);
+      }
+      if (M_dbg) {
+        float* md = M_dbg + (size_t)m * kDD + (size_t)i * kD + 32 * q;
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) md[c2] = -__uint_as_float(v[c2]);
+      }
+    }
+    // the next matrix overwrites these TMEM rows: every lane's reads first
+    tc_fence_before();
+    named_bar_sync(bid, 128);
+    tc_fence_after();
+  }
+  if (i == 0) {   // the group's own tensor-core work completes before TMEM is released
+    mma_commit(sbar);
+    mbar_wait_drain(sbar, sweep_phase);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -394,22 +566,38 @@ k_sweep_inverse_img(const float* __restrict__ A, uint8_t* __restrict__ Mimg, flo
 // Step t: X = S + B_t (fp32), then S <- X M_t computed on the tensor cores as
 //   D[j][n] = sum_k M[k][j] X[n][k]  with  M = Mh + Ml,  X = Xh + Xl  (bf16)
 //   D = Mh Xh + Mh Xl + Ml Xh        (the dropped Ml Xl term is ~2^-16 rel.)
-// TMEM lane j holds column j of S (all 128 rows n in columns 0..127).
-// Warps 0-3: state (thread j = TMEM lane j): read S from TMEM, store boundary
-// states, add B_{t+1} (prefetched into registers), write the X hi/lo image
-// (K-major, 128-B swizzle).  Warp 4: bulk-copies the M image of the coming
-// steps (two stages).  Warp 5: MMA issuer, TMEM owner.
+// Right-multiplication acts on each row of S independently, so the 128 rows
+// run as two independent 64-row halves that ping-pong: while the tensor pipe
+// works on one half, the state warps rebuild the other half's operand, and
+// the pipe always has the next half queued.  TMEM: half h in columns
+// 64h .. 64h+63; lane j holds column j of S.
+// Warps 0-7: state; warps 4h .. 4h+3 own half h (thread j = TMEM lane j of
+// its quarter): read S from TMEM, store boundary states, add B_{t+1}
+// (prefetched into registers), write the X hi/lo image (K-major, 128-B
+// swizzle, one 16 KB image per half and per hi/lo).  The two halves' operand
+// rebuilds run on separate warps, so the tensor pipe sets the step time.
+// Warp 8: bulk-copies the M image of the coming steps (two stages).
+// Warp 9: MMA issuer, TMEM owner.
 // Boundary states: fwd[j] after frames [0, jC), rev[j] after [jC, T).
 // ===========================================================================
 struct ScanCfg {
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
+  static constexpr int PREFETCH = 3;                       // steps of L2 prefetch lead
+  static constexpr int WARP_PROD = 8;
+  static constexpr int WARP_MMA = 9;
   static constexpr uint32_t OFF_M = 0;                    // 2 stages x 64 KB
-  static constexpr uint32_t OFF_X = 2 * kImgBytes;        // X hi (32 KB) + lo (32 KB)
+  static constexpr uint32_t OFF_X = 2 * kImgBytes;        // [half][hi/lo] x 16 KB
+  static constexpr uint32_t XIMG = 16384;                 // 64 rows x 128 k bf16
   static constexpr uint32_t BAR_OFF = 3 * kImgBytes;
-  static constexpr int NBAR = 2 + 2 + 1 + 1 + 1;           // mfull[2], mempty[2], xfull, dfull, drain
+  static constexpr int NBAR = 2 + 2 + 2 + 2 + 1;           // mfull[2], mempty[2], xfull[2], dfull[2], drain
   static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
 };
 
+// X image of one 64-row half: element (n, k), n < 64: k-block (k / 64) of
+// 64 rows x 128 B, 128-B swizzle
+__device__ __forceinline__ uint32_t ximg64_offset(int n, int k) {
+  return (uint32_t)(k >> 6) * 8192u + sw128_offset((uint32_t)n, (uint32_t)(k & 63));
+}
 __device__ __forceinline__ uint32_t ximg_offset(int n, int k) {
   return (uint32_t)(k >> 6) * 16384u + sw128_offset((uint32_t)n, (uint32_t)(k & 63));
 }
@@ -423,7 +611,7 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
   auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
-  const int MFULL = 0, MEMPTY = 2, XFULL = 4, DFULL = 5, DRAIN = 6;
+  const int MFULL = 0, MEMPTY = 2, XFULL = 4, DFULL = 6, DRAIN = 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -433,14 +621,14 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(MFULL + s), 1);
       mbar_init(BAR(MEMPTY + s), 1);
+      mbar_init(BAR(XFULL + s), 128);
+      mbar_init(BAR(DFULL + s), 1);
     }
-    mbar_init(BAR(XFULL), 128);
-    mbar_init(BAR(DFULL), 1);
     mbar_init(BAR(DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == C::WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), 128);
     tmem_relinquish();
   }
@@ -451,7 +639,7 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
   auto frame_of = [&](int i) { return dir == 0 ? i : T - 1 - i; };
   int last_i[2] = {-1, -1};   // producer: last step issued on each stage
 
-  if (warp == 4) {
+  if (warp == C::WARP_PROD) {
     // ---------------- M image producer
     if (lane == 0) {
       for (int i = 0; i < T; ++i) {
@@ -460,75 +648,83 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
         mbar_arrive_expect_tx(BAR(MFULL + s), kImgBytes);
         const uint8_t* src = Mimg + ((size_t)bh * T + frame_of(i)) * kImgBytes;
         const uint32_t dst = sbase + C::OFF_M + s * kImgBytes;
+        if (i + C::PREFETCH < T) {   // warm L2 with the M image and B of a later step
+          const size_t fa = (size_t)bh * T + frame_of(i + C::PREFETCH);
+          bulk_prefetch_l2(Mimg + fa * kImgBytes, kImgBytes);
+          bulk_prefetch_l2(Bm + fa * kDD, (uint32_t)(kDD * sizeof(float)));
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) bulk_load(dst + q * 16384u, src + q * 16384u, 16384u, BAR(MFULL + s));
         last_i[s] = i;
       }
     }
-  } else if (warp == 5) {
-    // ---------------- MMA issuer
+  } else if (warp == C::WARP_MMA) {
+    // ---------------- MMA issuer: step i = half 0, then half 1
     if (lane == 0) {
-      constexpr uint32_t kId = idesc_bf16(128, 128, 1, 0);   // A (M image) MN-major, B (X) K-major
-      const uint32_t xh = sbase + C::OFF_X, xl = xh + kImgHalf;
-      for (int i = 0; i < T; ++i) {
+      constexpr uint32_t kId = idesc_bf16(128, 64, 1, 0);   // A (M image) MN-major, B (X half) K-major
+      bool ok = true;
+      for (int i = 0; ok && i < T; ++i) {
         const uint32_t s = (uint32_t)i & 1u, ph = ((uint32_t)i >> 1) & 1u;
-        if (!mbar_wait(BAR(XFULL), (uint32_t)i & 1u, abort_flag)) break;
         if (!mbar_wait(BAR(MFULL + s), ph, abort_flag)) break;
-        tc_fence_after();
         const uint32_t mh = sbase + C::OFF_M + s * kImgBytes, ml = mh + kImgHalf;
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(BAR(XFULL + h), (uint32_t)i & 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t xh = sbase + C::OFF_X + (uint32_t)h * 2u * C::XIMG, xl = xh + C::XIMG;
+          const uint32_t d = tmem + 64u * (uint32_t)h;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t ao = (uint32_t)ks * 2048u;                              // 16 k-rows
-          const uint32_t bo = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;  // 16 k-columns
-          const uint64_t a_h = desc_sw128(mh + ao, 16384, 1024), a_l = desc_sw128(ml + ao, 16384, 1024);
-          const uint64_t b_h = desc_sw128(xh + bo, 16, 1024), b_l = desc_sw128(xl + bo, 16, 1024);
-          mma_bf16_ss(tmem, a_h, b_h, kId, ks != 0);
-          mma_bf16_ss(tmem, a_h, b_l, kId, 1u);
-          mma_bf16_ss(tmem, a_l, b_h, kId, 1u);
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t ao = (uint32_t)ks * 2048u;                                  // 16 k-rows
+            const uint32_t bo = (uint32_t)(ks >> 2) * 8192u + (uint32_t)(ks & 3) * 32u;  // 16 k-columns
+            const uint64_t a_h = desc_sw128(mh + ao, 16384, 1024), a_l = desc_sw128(ml + ao, 16384, 1024);
+            const uint64_t b_h = desc_sw128(xh + bo, 16, 1024), b_l = desc_sw128(xl + bo, 16, 1024);
+            mma_bf16_ss(d, a_h, b_h, kId, ks != 0);
+            mma_bf16_ss(d, a_h, b_l, kId, 1u);
+            mma_bf16_ss(d, a_l, b_h, kId, 1u);
+          }
+          mma_commit(BAR(DFULL + h));
         }
-        mma_commit(BAR(MEMPTY + s));
-        mma_commit(BAR(DFULL));
+        if (ok) mma_commit(BAR(MEMPTY + s));
       }
       mma_commit(BAR(DRAIN));
       mbar_wait_drain(BAR(DRAIN), 0);
     }
     __syncwarp();
   } else {
-    // ---------------- state warps: thread j owns column j of S
-    const int j = warp * 32 + lane;
+    // ---------------- state warps: half h = warp / 4, thread j owns column j of S
+    const int h = warp >> 2, q = warp & 3;
+    const int j = q * 32 + lane;
     const float* S0 = dir == 0 ? S0f : S0r;
     float* st = states + ((size_t)dir * BH + bh) * (size_t)(NC + 1) * kDD;
-    uint8_t* xh = smem + C::OFF_X;
-    uint8_t* xl = xh + kImgHalf;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-    float bnext[kD];
+    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + 64u * (uint32_t)h;
+    // X image address of element (n2, j) = xs + n2 * 128 + xr[n2 & 7]
+    const uint32_t xs = sbase + C::OFF_X + (uint32_t)h * 2u * C::XIMG + (uint32_t)(j >> 6) * 8192u +
+                        (uint32_t)(j & 7) * 2u;
+    uint32_t xr[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) xr[r] = (uint32_t)((((j & 63) >> 3) ^ r) << 4);
+    float bnext[64];
 
     // initial state: store it as the first boundary, X_0 = S0 + B_{t0}
     {
       const int j0 = dir == 0 ? 0 : NC;
-      const float* B0 = Bm + ((size_t)bh * T + frame_of(0)) * kDD;
+      const float* B0 = Bm + ((size_t)bh * T + frame_of(0)) * kDD + (size_t)(64 * h) * kD + j;
 #pragma unroll 8
-      for (int n = 0; n < kD; ++n) {
+      for (int n2 = 0; n2 < 64; ++n2) {
+        const int n = 64 * h + n2;
         const float s0 = S0 ? __ldg(S0 + (size_t)bh * kDD + (size_t)n * kD + j) : 0.f;
         st[(size_t)j0 * kDD + (size_t)n * kD + j] = s0;
-        float h, l;
-        split_bf16(s0 + __ldg(B0 + (size_t)n * kD + j), h, l);
-        const uint32_t off = ximg_offset(n, j);
-        *reinterpret_cast<__nv_bfloat16*>(xh + off) = __float2bfloat16_rn(h);
-        *reinterpret_cast<__nv_bfloat16*>(xl + off) = __float2bfloat16_rn(l);
+        float hi, lo;
+        split_bf16(s0 + __ldg(B0 + (size_t)n2 * kD), hi, lo);
+        const uint32_t a = xs + (uint32_t)n2 * 128u + xr[n2 & 7];
+        st_shared_u16(a, bf16_bits(hi));
+        st_shared_u16(a + C::XIMG, bf16_bits(lo));
       }
       fence_proxy_async_smem();
-      mbar_arrive(BAR(XFULL));
+      mbar_arrive(BAR(XFULL + h));
     }
     for (int i = 0; i < T; ++i) {
       const bool more = i + 1 < T;
-      if (more) {
-        const float* Bn = Bm + ((size_t)bh * T + frame_of(i + 1)) * kDD;
-#pragma unroll
-        for (int n = 0; n < kD; ++n) bnext[n] = __ldg(Bn + (size_t)n * kD + j);
-      }
-      if (!__all_sync(0xffffffffu, mbar_wait(BAR(DFULL), (uint32_t)i & 1u, abort_flag))) break;
-      tc_fence_after();
       const int t = frame_of(i);
       int jb = -1;
       if (dir == 0) {
@@ -536,40 +732,47 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
       } else if (t % chunk == 0) {
         jb = t / chunk;
       }
+      if (more) {   // B_{t+1}[64h + n2][j]: 32 lanes read 128 contiguous bytes per row
+        const float* Bn = Bm + ((size_t)bh * T + frame_of(i + 1)) * kDD + (size_t)(64 * h) * kD + j;
+#pragma unroll
+        for (int n2 = 0; n2 < 64; ++n2) bnext[n2] = __ldg(Bn + (size_t)n2 * kD);
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(DFULL + h), (uint32_t)i & 1u, abort_flag))) break;
+      tc_fence_after();
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
-        uint32_t v[32];
-        tmem_ld32(trow + cb * 32, v);
+        uint32_t v[16];
+        tmem_ld16(trow + cb * 16, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int n = cb * 32 + c;
-          const float s = __uint_as_float(v[c]);
-          if (jb >= 0) st[(size_t)jb * kDD + (size_t)n * kD + j] = s;
+        for (int c = 0; c < 16; ++c) {
+          const int n2 = cb * 16 + c;
+          const float sv = __uint_as_float(v[c]);
+          if (jb >= 0) st[(size_t)jb * kDD + (size_t)(64 * h + n2) * kD + j] = sv;
           if (more) {
-            float h, l;
-            split_bf16(s + bnext[n], h, l);
-            const uint32_t off = ximg_offset(n, j);
-            *reinterpret_cast<__nv_bfloat16*>(xh + off) = __float2bfloat16_rn(h);
-            *reinterpret_cast<__nv_bfloat16*>(xl + off) = __float2bfloat16_rn(l);
+            float hi, lo;
+            split_bf16(sv + bnext[n2], hi, lo);
+            const uint32_t a = xs + (uint32_t)n2 * 128u + xr[c & 7];
+            st_shared_u16(a, bf16_bits(hi));
+            st_shared_u16(a + C::XIMG, bf16_bits(lo));
           }
         }
       }
       if (more) {
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(BAR(XFULL));
+        mbar_arrive(BAR(XFULL + h));
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == C::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 128);
   }
-  if (warp == 4 && lane == 0 && *abort_flag) {  // let issued copies land before the CTA exits
+  if (warp == C::WARP_PROD && lane == 0 && *abort_flag) {  // let issued copies land before the CTA exits
     for (int s = 0; s < 2; ++s)
       if (last_i[s] >= 0) mbar_wait_drain(BAR(MFULL + s), ((uint32_t)last_i[s] >> 1) & 1u);
   }
@@ -732,8 +935,8 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     // ---------------- epilogue (thread r = token row r of the tile) + S~ builder
     const int r = warp * 32 + lane;
     const uint32_t trow_base = tmem + ((uint32_t)(warp * 32) << 16);
-    uint8_t* simg_h = smem + C::OFF_S;
-    uint8_t* simg_l = simg_h + kImgHalf;
+    const uint32_t simg_s = sbase + C::OFF_S;
+    const uint32_t sw_s = sbase + C::OFF_W;
     int k = 0, prev_bh = -1, prev_c = -1;
     const size_t sdir = (size_t)g.BH * (size_t)(g.NC + 1) * kDD;
     for (long long gt = t_begin; gt < t_end; ++gt, ++k) {
@@ -763,8 +966,8 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             lw[q] = pack_bf16(l0, l1);
           }
           const uint32_t off = ximg_offset(r, cc * 8);   // row i = r, columns k = 8cc..8cc+7
-          *reinterpret_cast<uint4*>(simg_h + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(simg_l + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          st_shared_v4(simg_s + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+          st_shared_v4(simg_s + kImgHalf + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
         }
         fence_proxy_async_smem();
         mbar_arrive(BAR(SREADY));
@@ -798,15 +1001,15 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       for (int i = 0; i < kD; ++i) ss = fmaf(o[i], o[i], ss);
       const float rinv = rsqrtf(ss * (1.0f / kD) + eps);
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(GFULL + s), ph, abort_flag))) break;
-      const uint8_t* gt_s = smem + C::OFF_G + s * C::TILE_BYTES;
+      const uint32_t gt_s = sbase + C::OFF_G + s * C::TILE_BYTES;
       const bool valid = tr + r < rows;
       __nv_bfloat16* orow = out + ((size_t)bh * tokens_per_head + (size_t)c * g.chunk * g.U + tr + r) * kD;
 #pragma unroll
       for (int cc = 0; cc < 16; ++cc) {
         const uint32_t off = (uint32_t)(cc >> 3) * (C::TILE_BYTES / 2) + sw128_offset((uint32_t)r, (uint32_t)((cc & 7) * 8));
-        const uint4 gv = *reinterpret_cast<const uint4*>(gt_s + off);
-        const float4 wa = *reinterpret_cast<const float4*>(sw + cc * 8);
-        const float4 wb = *reinterpret_cast<const float4*>(sw + cc * 8 + 4);
+        const uint4 gv = ld_shared_v4(gt_s + off);
+        const float4 wa = ld_shared_f4(sw_s + (uint32_t)cc * 32u);
+        const float4 wb = ld_shared_f4(sw_s + (uint32_t)cc * 32u + 16u);
         const float wh[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
         const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
         uint32_t yw[4];
@@ -928,6 +1131,8 @@ inline int num_sms() {
 }
 
 // frame statistics for FH frame-heads of U tokens (K, V: [FH][U][128] bf16)
+// Statistics for FH frame-heads of U tokens (K, V: [FH][U][128] bf16):
+// A [FH][d_k][d_k] and B [FH][d_v][d_k], fp32.
 inline int launch_stats(const void* K, const void* V, const float* beta, int U, size_t FH, float* A, float* B,
                         cudaStream_t s) {
   CUtensorMap tmK, tmV;
@@ -935,15 +1140,21 @@ inline int launch_stats(const void* K, const void* V, const float* beta, int U, 
     return VDA_ERR_CUDA;
   if (cudaFuncSetAttribute(k_stats_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StatsCfg::SMEM) !=
       cudaSuccess)
-    return VDA_ERR_CUDA;
+    return launch_status("k_stats_tc (shared-memory attribute)");
   const int grid = (int)std::min<size_t>(FH, (size_t)num_sms());
   k_stats_tc<<<grid, StatsCfg::THREADS, StatsCfg::SMEM, s>>>(tmK, tmV, beta, U, (int)FH, A, B);
   return launch_status("k_stats_tc");
 }
 
-inline int launch_inverse_img(const float* A, uint8_t* Mimg, float* M_f32, size_t FH, cudaStream_t s) {
-  k_sweep_inverse_img<<<(unsigned)FH, kSweepThreads, 0, s>>>(A, Mimg, M_f32);
-  return launch_status("k_sweep_inverse_img");
+// M = (I + A)^{-1} images (and optional fp32 copy) for FH matrices
+inline int launch_inverse(const float* A, size_t FH, uint8_t* Mimg, float* M_dbg, cudaStream_t s) {
+  if (cudaFuncSetAttribute(k_inverse_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)InvCfg::SMEM) !=
+      cudaSuccess)
+    return launch_status("k_inverse_tc (shared-memory attribute)");
+  const size_t per_cta = (size_t)InvCfg::GROUPS;
+  const int grid = (int)std::min<size_t>((FH + per_cta - 1) / per_cta, (size_t)num_sms());
+  k_inverse_tc<<<grid, InvCfg::THREADS, InvCfg::SMEM, s>>>(A, (int)FH, Mimg, M_dbg);
+  return launch_status("k_inverse_tc");
 }
 
 inline int launch_scan(const uint8_t* Mimg, const float* Bm, const float* S0f, const float* S0r, float* states,
@@ -986,6 +1197,7 @@ inline int launch_readout(const void* Q, const void* G, const float* w, const fl
 inline bool tc_path_supported(int d, int dtype) { return d == 128 && dtype == VDA_BF16; }
 
 // extra workspace of the tensor-core path: the M hi/lo operand images
+// (64 KB per frame-head), next to A
 inline size_t tc_extra_workspace_bytes(bool tc, size_t FH, int d) {
   (void)d;
   return tc ? FH * (size_t)tc::kImgBytes : 0;
@@ -999,23 +1211,22 @@ int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_
   const size_t FH = BH * (size_t)T;
   const size_t fdd = FH * tc::kDD;
   float* A = reinterpret_cast<float*>(ws_AM);
-  float* Bm = reinterpret_cast<float*>(ws_B);
+  float* Bt = reinterpret_cast<float*>(ws_B);
   float* st = reinterpret_cast<float*>(ws_states);
   uint8_t* img = reinterpret_cast<uint8_t*>(ws_img);
   int rc;
   mark(0);
-  if ((rc = tc::launch_stats(a.k, a.v, a.beta, U, FH, A, Bm, s)) != VDA_OK) return rc;
+  if ((rc = tc::launch_stats(a.k, a.v, a.beta, U, FH, A, Bt, s)) != VDA_OK) return rc;
   if ((rc = debug_check("stats", s)) != VDA_OK) return rc;
-  if (stats_out) {
-    if (cudaMemcpyAsync(stats_out, A, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(stats_out + fdd, Bm, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
-      return VDA_ERR_CUDA;
-  }
+  if (stats_out &&
+      (cudaMemcpyAsync(stats_out, A, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+       cudaMemcpyAsync(stats_out + fdd, Bt, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess))
+    return VDA_ERR_CUDA;
   mark(1);
-  if ((rc = tc::launch_inverse_img(A, img, stats_out ? stats_out + 2 * fdd : nullptr, FH, s)) != VDA_OK) return rc;
+  if ((rc = tc::launch_inverse(A, FH, img, stats_out ? stats_out + 2 * fdd : nullptr, s)) != VDA_OK) return rc;
   if ((rc = debug_check("inverse", s)) != VDA_OK) return rc;
   mark(2);
-  if ((rc = tc::launch_scan(img, Bm, a.S0_fwd, a.S0_rev, st, BH, T, chunk, NC, 2, s)) != VDA_OK) return rc;
+  if ((rc = tc::launch_scan(img, Bt, a.S0_fwd, a.S0_rev, st, BH, T, chunk, NC, 2, s)) != VDA_OK) return rc;
   if ((rc = debug_check("scan", s)) != VDA_OK) return rc;
   mark(3);
   const float eps = a.eps > 0.f ? a.eps : 1e-6f;
@@ -1032,12 +1243,12 @@ int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_
 inline int tc_text_state(size_t BH, int L, const void* k, const void* v, const float* beta, char* ws_AM,
                          char* ws_B, char* ws_states, char* ws_img, cudaStream_t s) {
   float* A = reinterpret_cast<float*>(ws_AM);
-  float* Bm = reinterpret_cast<float*>(ws_B);
+  float* Bt = reinterpret_cast<float*>(ws_B);
   uint8_t* img = reinterpret_cast<uint8_t*>(ws_img);
   int rc;
-  if ((rc = tc::launch_stats(k, v, beta, L, BH, A, Bm, s)) != VDA_OK) return rc;
-  if ((rc = tc::launch_inverse_img(A, img, nullptr, BH, s)) != VDA_OK) return rc;
-  return tc::launch_scan(img, Bm, nullptr, nullptr, reinterpret_cast<float*>(ws_states), BH, 1, 1, 1, 1, s);
+  if ((rc = tc::launch_stats(k, v, beta, L, BH, A, Bt, s)) != VDA_OK) return rc;
+  if ((rc = tc::launch_inverse(A, BH, img, nullptr, s)) != VDA_OK) return rc;
+  return tc::launch_scan(img, Bt, nullptr, nullptr, reinterpret_cast<float*>(ws_states), BH, 1, 1, 1, 1, s);
 }
 
 }  // namespace vda
