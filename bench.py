@@ -156,11 +156,17 @@ def algorithmic(wl):
     }
 
 
-STAGE_BOUND = {"stats": "hbm", "inverse": "alu", "scan": "hbm", "readout": "hbm"}
-STAGE_KERNEL = {"stats": ("k_stats", ["kernels_simt.cuh", "kernels_tc.cuh"]),
-                "inverse": ("k_gj_inverse", ["kernels_simt.cuh"]),
-                "scan": ("k_scan", ["kernels_simt.cuh", "kernels_tc.cuh"]),
-                "readout": ("k_readout", ["kernels_simt.cuh", "kernels_tc.cuh"])}
+def stage_kernels(wl):
+    """(bound, kernel name, source files) of each stage's kernel on the path
+    the library takes for this workload: tensor cores for bf16 I/O at
+    d_k = d_v = 128, the SIMT kernels otherwise."""
+    if wl.dtype == "bf16" and wl.d == 128:
+        src = ["kernels_tc.cuh", "tc_ptx.cuh"]
+        return {"stats": ("hbm", "k_stats_tc", src), "inverse": ("hbm", "k_inverse_tc", src),
+                "scan": ("hbm", "k_scan_tc", src), "readout": ("hbm", "k_readout_tc", src)}
+    src = ["kernels_simt.cuh"]
+    return {"stats": ("hbm", "k_stats_simt", src), "inverse": ("alu", "k_gj_inverse", src),
+            "scan": ("hbm", "k_scan_simt", src), "readout": ("hbm", "k_readout_simt", src)}
 
 
 def fp32_alu_peak_tflops(sm_mhz):
@@ -375,7 +381,7 @@ def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches):
     alg = algorithmic(wl)
     dom = max(stage_ms, key=stage_ms.get)
     dom_ms = stage_ms[dom] / max(calls, 1)
-    bound = STAGE_BOUND[dom]
+    bound, kname, _ = stage_kernels(wl)[dom]
     sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
     if bound == "hbm":
         achieved = alg[dom]["bytes"] / (dom_ms * 1e-3) / 1e9
@@ -385,7 +391,6 @@ def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches):
         achieved = alg[dom]["flops"] / (dom_ms * 1e-3) / 1e12
         peak, unit = fp32_alu_peak_tflops(sm_mhz), "TFLOP/s"
         peak_note = f"FP32 FMA peak 148 SMs x 128 lanes x 2 at the sampled {sm_mhz:.0f} MHz"
-    kname, ksrc = STAGE_KERNEL[dom]
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": recorded_traffic(kname), "kernel": kname, "stage": dom,
                 "kernel_ms": dom_ms, "algorithmic_per_launch": alg[dom]["bytes" if bound == "hbm" else "flops"],

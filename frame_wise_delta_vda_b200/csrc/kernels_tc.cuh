@@ -300,126 +300,168 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
 // k_inverse_tc: M = (I + A)^{-1} for every frame-head, by a block sweep of the
 // symmetric positive definite I + A held in TMEM, with the rank-16 updates
 // on the tensor cores.  Sweeping every index of a symmetric matrix ends at
-// its negative inverse; with pivot blocks P = [16K, 16K + 16), one block step
-//   G = -P^{-1}                 (16 x 16 sweep with warp shuffles)
+// its negative inverse; with pivot blocks P of 16 indices, one block step
+//   G = -P^{-1}                 (16 x 16 sweep in one warp)
 //   A_ij += (C G)_i C_j^T       (i, j outside P; C = A[:, P]; one MMA)
 //   A_iP = W_i = -(C G)_i,  A_PP = G,  A_Pj = W_j^T   (fix-ups)
 // sweeps the 16 indices of P at once.  Every pivot block of an SPD matrix's
-// Schur complement is SPD, so no pivoting is needed.  C, G and C G go to the
-// tensor cores as bf16 hi + lo (three products, ~16 significant bits).
-// Three warpgroups per CTA work on three matrices at once (own TMEM
-// columns, shared-memory workspace, named barrier and completion barrier),
-// so their round trips to the tensor pipe interleave.  In: A rows (fp32, from
+// Schur complement is SPD, so no pivoting is needed.  C G is formed on the
+// CUDA cores in fp32; C and C G go to the tensor cores as bf16 hi + lo (three
+// products, ~16 significant bits).  The 16 x 16 sweep is the sequential part,
+// so it runs one block ahead: while the tensor cores update the matrix with
+// block P, the warp owning the next block Q brings A_QQ up to date itself
+// (A_QQ + (C G)_Q C_Q^T in fp32) and sweeps it.  Three warpgroups per CTA
+// work on three matrices at once (own TMEM columns, shared-memory workspace,
+// named barrier and completion barrier).  In: A rows (fp32, from
 // k_stats_tc).  Out: the scan's M operand image (element (j, k) = M[k][j],
 // MN-major, 128-B swizzle, bf16 hi / lo halves) and optionally M in fp32.
 // ===========================================================================
 struct InvCfg {
   static constexpr int GROUPS = 3;
   static constexpr int THREADS = 128 * GROUPS;
-  static constexpr uint32_t TCOLS = 160;     // TMEM columns per group: A (128) + C G scratch (16)
-  static constexpr uint32_t SW_BYTES = 25728; // per-group workspace (see SW_* below)
+  static constexpr uint32_t TCOLS = 128;     // TMEM columns per group: the matrix
+  static constexpr uint32_t SW_BYTES = 28672; // per-group workspace (see SW_* below)
   static constexpr uint32_t BAR_OFF = GROUPS * SW_BYTES;
   static constexpr size_t SMEM = BAR_OFF + GROUPS * 8 + 16 + 1024;
 };
 // per-group workspace: K-major no-swizzle operand images (rows of 16 bf16)
+// and fp32 exchange buffers
 constexpr uint32_t SW_CH = 0, SW_CL = 4096;        // panel C, 128 rows
-constexpr uint32_t SW_GH = 8192, SW_GL = 8704;     // G = -P^{-1}, 16 rows
-constexpr uint32_t SW_CGH = 9216, SW_CGL = 13312;  // C G, 128 rows
-constexpr uint32_t SW_W = 17408;                   // W^T = (-C G)^T, fp32 [16][128]
-constexpr uint32_t SW_PB = 25600;                  // pivot-row broadcast, fp32 [2][16]
+constexpr uint32_t SW_CGH = 8192, SW_CGL = 12288;  // C G, 128 rows
+constexpr uint32_t SW_W = 16384;                   // W^T = (-C G)^T, [16][128]
+constexpr uint32_t SW_G = 24576;                   // G = -P^{-1}, [2 buffers][16][16]
+constexpr uint32_t SW_CQ = 26624;                  // next block's rows of C, transposed, [2 segments][16][16]
+
+// Pivot block swept at step s by group grp: the order 0,2,4,6,1,3,5,7 rotated
+// by grp.  The sweep's result does not depend on the order; this one puts
+// consecutive blocks in different warps (a block's TMEM lanes belong to warp
+// block / 2, i.e. to a fixed sub-partition) and the groups' pivot warps of
+// one step on different sub-partitions.
+__device__ __forceinline__ int inv_block(int s, int grp) {
+  const int j = (s + grp) & 7;
+  return j < 4 ? 2 * j : 2 * j - 7;
+}
+
+// In-place sweep of a symmetric 16 x 16 block by one warp.  On entry the
+// block's rows are in the 16-lane segment `sel` (row r = lane & 15, all 16
+// columns in x); on exit every lane holds row r, columns [8h, 8h + 8) of
+// -P^{-1} in g (h = lane >> 4), so both segments share the arithmetic.  The
+// pivot row and the pivot column element come from the owning lanes by
+// shuffles.
+__device__ __forceinline__ void sweep16(const float (&x)[16], int sel, int lane, float (&g)[8]) {
+  const int r = lane & 15, h = lane >> 4;
+  const int src = r + 16 * sel;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const float a = __shfl_sync(0xffffffffu, x[t], src);
+    const float b = __shfl_sync(0xffffffffu, x[8 + t], src);
+    g[t] = h ? b : a;
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int kh = k >> 3, kk = k & 7;
+    float col[8];   // row k at this lane's columns
+#pragma unroll
+    for (int t = 0; t < 8; ++t) col[t] = __shfl_sync(0xffffffffu, g[t], k + 16 * h);
+    const float akk = __shfl_sync(0xffffffffu, g[kk], k + 16 * kh);   // pivot
+    const float ark = __shfl_sync(0xffffffffu, g[kk], r + 16 * kh);   // this row's column k
+    const float pinv = rcp_approx(akk);
+    const bool me = r == k;
+    const float f = ark * pinv;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) g[t] = me ? col[t] * pinv : fmaf(-f, col[t], g[t]);
+    if (h == kh) g[kk] = me ? -pinv : f;
+  }
+}
+
+__device__ __forceinline__ void st_row8_f32(uint32_t addr, const float (&x)[8]) {
+#pragma unroll
+  for (int t = 0; t < 8; t += 4)
+    st_shared_v4(addr + 4u * t, make_uint4(__float_as_uint(x[t]), __float_as_uint(x[t + 1]),
+                                           __float_as_uint(x[t + 2]), __float_as_uint(x[t + 3])));
+}
 
 // One warpgroup sweeps the matrix in TMEM columns [tA, tA + 128); thread i =
-// TMEM lane i; gw = warp index within the group.  Returns false on abort.
-__device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t tW, uint32_t lb, uint32_t swb,
-                                                   uint32_t bid, uint32_t sbar, uint32_t& sweep_phase,
-                                                   volatile int* abort_flag, int i, int gw, int lane) {
-  constexpr uint32_t kId16 = idesc_bf16(128, 16, 0, 0);
+// TMEM lane i; gw = warp index within the group, grp = group index.  bid:
+// the group's named barrier; bend: a second one that closes each step, so a
+// warp that only arrives at bid cannot reach bid again before every thread
+// has passed it.  Returns false on abort.
+__device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t lb, uint32_t swb, uint32_t bid,
+                                                   uint32_t bend, uint32_t sbar, uint32_t& sweep_phase,
+                                                   volatile int* abort_flag, int i, int gw, int lane, int grp) {
   constexpr uint32_t kId128 = idesc_bf16(128, 128, 0, 0);
-  bool ok = true;
-  // block sweep of I + A, pivot blocks P = [16K, 16K + 16):
-  //   G = -P^{-1} (16 x 16 sweep in the half-warp owning the rows of P),
-  //   C = A[:, P], A += (C G) C^T on the tensor cores (3-product bf16
-  //   split, into A's own TMEM columns), then the pivot columns become
-  //   W = -C G (G on the pivot rows) and the pivot rows W^T.  After all
-  //   eight blocks TMEM holds -(I + A)^{-1}.
+  const int r = lane & 15, h = lane >> 4;
+  const uint32_t cqb = swb + SW_CQ + (uint32_t)h * 1024u;
+  // G of the first pivot block (the matrix is untouched: P = its own block)
+  {
+    const int K0 = inv_block(0, grp);
+    if (gw == (K0 >> 1)) {
+      uint32_t v[16];
+      tmem_ld16(lb + tA + 16u * (uint32_t)K0, v);
+      tmem_wait_ld();
+      const bool in0 = (i >> 4) == K0;
+      float x0[16], g0[8];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) x0[t] = __uint_as_float(v[t]) + ((in0 && r == t) ? 1.f : 0.f);
+      sweep16(x0, K0 & 1, lane, g0);
+      st_row8_f32(swb + SW_G + 64u * (uint32_t)r + 32u * (uint32_t)h, g0);
+    }
+    named_bar_sync(bid, 128);
+  }
 #pragma unroll 1
-  for (int K = 0; K < 8; ++K) {
+  for (int s = 0; s < 8; ++s) {
+    const int K = inv_block(s, grp);
     const uint32_t p0 = 16u * (uint32_t)K;
     const bool inP = (i >> 4) == K;
     const bool pwarp = gw == (K >> 1);
-    float c[16];
+    const int Kn = inv_block(s + 1, grp);
+    const bool qwarp = s < 7 && gw == (Kn >> 1);     // sweeps the next block ahead
+    const bool inQ = qwarp && (i >> 4) == Kn;
+    const uint32_t gcur = swb + SW_G + 1024u * (uint32_t)(s & 1);
+    const uint32_t gnext = swb + SW_G + 1024u * (uint32_t)((s + 1) & 1);
+    // panel C (identity on P's diagonal); the next block's columns for its warp
+    float c[16], aq[16];
     {
       uint32_t v[16];
       tmem_ld16(lb + tA + p0, v);
-      tmem_wait_ld();
+      if (qwarp) {
+        uint32_t w2[16];
+        tmem_ld16(lb + tA + 16u * (uint32_t)Kn, w2);
+        tmem_wait_ld();
 #pragma unroll
-      for (int t = 0; t < 16; ++t)
-        c[t] = __uint_as_float(v[t]) + ((inP && (i & 15) == t) ? 1.f : 0.f);   // identity on P's diagonal
-    }
-    float g[16];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) g[t] = c[t];
-    if (pwarp) {   // 16 x 16 sweep per 16-lane segment (the segment owning P is used)
-      const int r = lane & 15;
-      const uint32_t pb = swb + SW_PB + (uint32_t)(lane >> 4) * 64u;   // this segment's broadcast row
-#pragma unroll
-      for (int sidx = 0; sidx < 16; ++sidx) {
-        // row sidx = column sidx (symmetric): its owner publishes it for the segment
-        if (r == sidx) {
-#pragma unroll
-          for (int t = 0; t < 16; t += 4)
-            st_shared_v4(pb + 4u * t, make_uint4(__float_as_uint(g[t]), __float_as_uint(g[t + 1]),
-                                                 __float_as_uint(g[t + 2]), __float_as_uint(g[t + 3])));
-        }
-        __syncwarp();
-        float col[16];
-#pragma unroll
-        for (int t = 0; t < 16; t += 4) {
-          const float4 x = ld_shared_f4(pb + 4u * t);
-          col[t] = x.x; col[t + 1] = x.y; col[t + 2] = x.z; col[t + 3] = x.w;
-        }
-        __syncwarp();
-        const float pinv = rcp_approx(col[sidx]);
-        const bool me = r == sidx;
-        const float f = g[sidx] * pinv;
-#pragma unroll
-        for (int t = 0; t < 16; ++t) g[t] = me ? col[t] * pinv : fmaf(-f, col[t], g[t]);
-        g[sidx] = me ? -pinv : f;
+        for (int t = 0; t < 16; ++t) aq[t] = __uint_as_float(w2[t]) + ((inQ && r == t) ? 1.f : 0.f);
+      } else {
+        tmem_wait_ld();
       }
-      if (inP) store_row16_hilo(swb + SW_GH, swb + SW_GL, (uint32_t)r, g);
+#pragma unroll
+      for (int t = 0; t < 16; ++t) c[t] = __uint_as_float(v[t]) + ((inP && r == t) ? 1.f : 0.f);
+    }
+    // C G in fp32 (G symmetric, broadcast from shared memory)
+    float cg[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) cg[t] = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+#pragma unroll
+      for (int t = 0; t < 16; t += 4) {
+        const float4 x = ld_shared_f4(gcur + 64u * (uint32_t)k + 4u * t);
+        cg[t] = fmaf(c[k], x.x, cg[t]); cg[t + 1] = fmaf(c[k], x.y, cg[t + 1]);
+        cg[t + 2] = fmaf(c[k], x.z, cg[t + 2]); cg[t + 3] = fmaf(c[k], x.w, cg[t + 3]);
+      }
     }
     store_row16_hilo(swb + SW_CH, swb + SW_CL, (uint32_t)i, c);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    named_bar_sync(bid, 128);
-    if (i == 0) {   // C G -> scratch columns [128, 144) of this buffer
-      tc_fence_after();
-      const uint64_t ch = desc_noswz(swb + SW_CH, 128, 256), cl = desc_noswz(swb + SW_CL, 128, 256);
-      const uint64_t gh = desc_noswz(swb + SW_GH, 128, 256), gl = desc_noswz(swb + SW_GL, 128, 256);
-      mma_bf16_ss(tW, ch, gh, kId16, 0u);
-      mma_bf16_ss(tW, ch, gl, kId16, 1u);
-      mma_bf16_ss(tW, cl, gh, kId16, 1u);
-      mma_commit(sbar);
-    }
-    ok = named_bar_and(bid, 128, mbar_wait(sbar, sweep_phase, abort_flag));
-    sweep_phase ^= 1u;
-    if (!ok) return false;
-    tc_fence_after();
-    float cg[16];
-    {
-      uint32_t v[16];
-      tmem_ld16(lb + tW, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int t = 0; t < 16; ++t) cg[t] = __uint_as_float(v[t]);
-    }
     store_row16_hilo(swb + SW_CGH, swb + SW_CGL, (uint32_t)i, cg);
 #pragma unroll
     for (int t = 0; t < 16; ++t)   // W^T[t][i] = -(C G)[i][t]; lanes write consecutive words
       st_shared_f1(swb + SW_W + (uint32_t)t * 512u + 4u * (uint32_t)i, -cg[t]);
+    if (qwarp) {   // C's rows of the next block, transposed: cq[k][r] = C[Q_r][k]
+#pragma unroll
+      for (int k = 0; k < 16; ++k) st_shared_f1(cqb + 64u * (uint32_t)k + 4u * (uint32_t)r, c[k]);
+    }
     fence_proxy_async_smem();
     tc_fence_before();
-    named_bar_sync(bid, 128);
+    if (qwarp && gw != 0) named_bar_arrive(bid, 128);
+    else named_bar_sync(bid, 128);
     if (i == 0) {   // A += (C G) C^T
       tc_fence_after();
       const uint64_t ch = desc_noswz(swb + SW_CH, 128, 256), cl = desc_noswz(swb + SW_CL, 128, 256);
@@ -429,46 +471,72 @@ __device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t tW, uin
       mma_bf16_ss(tA, ql, ch, kId128, 1u);
       mma_commit(sbar);
     }
-    ok = named_bar_and(bid, 128, mbar_wait(sbar, sweep_phase, abort_flag));
-    sweep_phase ^= 1u;
-    if (!ok) return false;
-    tc_fence_after();
-    // (3) fix-ups of the pivot columns (all rows) and pivot rows
-    if (pwarp) {   // rewrite the full rows of this warp's 32 lanes
-      const int r = lane & 15;
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        uint32_t v[32];
-        tmem_ld32(lb + tA + 32u * q, v);
-        tmem_wait_ld();
-        if (inP) {   // pivot rows: W_j^T for the columns outside P
+    if (qwarp) {   // next block after this step, A_QQ + (C G)_Q C_Q^T, and its sweep
+      __syncwarp();
 #pragma unroll
-          for (int t = 0; t < 32; t += 4) {
-            const float4 x = ld_shared_f4(swb + SW_W + (uint32_t)r * 512u + 4u * (uint32_t)(32 * q + t));
-            v[t] = __float_as_uint(x.x); v[t + 1] = __float_as_uint(x.y);
-            v[t + 2] = __float_as_uint(x.z); v[t + 3] = __float_as_uint(x.w);
-          }
+      for (int k = 0; k < 16; ++k) {
+#pragma unroll
+        for (int t = 0; t < 16; t += 4) {
+          const float4 x = ld_shared_f4(cqb + 64u * (uint32_t)k + 4u * t);
+          aq[t] = fmaf(cg[k], x.x, aq[t]); aq[t + 1] = fmaf(cg[k], x.y, aq[t + 1]);
+          aq[t + 2] = fmaf(cg[k], x.z, aq[t + 2]); aq[t + 3] = fmaf(cg[k], x.w, aq[t + 3]);
         }
-        if (q == (K >> 1)) {   // the 16 pivot columns sit in this 32-column chunk
-          if ((K & 1) == 0) {
-#pragma unroll
-            for (int t = 0; t < 16; ++t) v[t] = __float_as_uint(inP ? g[t] : -cg[t]);
-          } else {
-#pragma unroll
-            for (int t = 0; t < 16; ++t) v[16 + t] = __float_as_uint(inP ? g[t] : -cg[t]);
-          }
-        }
-        tmem_st32(lb + tA + 32u * q, v);
       }
-    } else {
-      uint32_t v[16];
-#pragma unroll
-      for (int t = 0; t < 16; ++t) v[t] = __float_as_uint(-cg[t]);
-      tmem_st16(lb + tA + p0, v);
+      float gq[8];
+      sweep16(aq, Kn & 1, lane, gq);
+      st_row8_f32(gnext + 64u * (uint32_t)r + 32u * (uint32_t)h, gq);
     }
-    tmem_wait_st();
+    bool ok = mbar_wait(sbar, sweep_phase, abort_flag);
+    sweep_phase ^= 1u;
+    tc_fence_after();
+    if (ok) {   // fix-ups of the pivot columns (all rows) and pivot rows
+      if (pwarp) {   // rewrite the full rows of this warp's 32 lanes
+        float gr[16];
+        if (inP) {
+#pragma unroll
+          for (int t = 0; t < 16; t += 4) {
+            const float4 x = ld_shared_f4(gcur + 64u * (uint32_t)r + 4u * t);
+            gr[t] = x.x; gr[t + 1] = x.y; gr[t + 2] = x.z; gr[t + 3] = x.w;
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 16; ++t) gr[t] = -cg[t];
+        }
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t v[32];
+          tmem_ld32(lb + tA + 32u * q, v);
+          tmem_wait_ld();
+          if (inP) {   // pivot rows: W_j^T for the columns outside P
+#pragma unroll
+            for (int t = 0; t < 32; t += 4) {
+              const float4 x = ld_shared_f4(swb + SW_W + (uint32_t)r * 512u + 4u * (uint32_t)(32 * q + t));
+              v[t] = __float_as_uint(x.x); v[t + 1] = __float_as_uint(x.y);
+              v[t + 2] = __float_as_uint(x.z); v[t + 3] = __float_as_uint(x.w);
+            }
+          }
+          if (q == (K >> 1)) {   // the 16 pivot columns sit in this 32-column chunk
+            if ((K & 1) == 0) {
+#pragma unroll
+              for (int t = 0; t < 16; ++t) v[t] = __float_as_uint(gr[t]);
+            } else {
+#pragma unroll
+              for (int t = 0; t < 16; ++t) v[16 + t] = __float_as_uint(gr[t]);
+            }
+          }
+          tmem_st32(lb + tA + 32u * q, v);
+        }
+      } else {
+        uint32_t v[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) v[t] = __float_as_uint(-cg[t]);
+        tmem_st16(lb + tA + p0, v);
+      }
+      tmem_wait_st();
+    }
     tc_fence_before();
-    named_bar_sync(bid, 128);
+    ok = named_bar_and(bend, 128, ok);
+    if (!ok) return false;
     tc_fence_after();
   }
   return true;
@@ -499,7 +567,7 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tA = tmem + C::TCOLS * (uint32_t)g, tW = tA + 128u;
+  const uint32_t tA = tmem + C::TCOLS * (uint32_t)g;
   const uint32_t lb = (uint32_t)(gw * 32) << 16;
   const uint32_t swb = sbase + C::SW_BYTES * (uint32_t)g;
   const uint32_t bid = 1u + (uint32_t)g;
@@ -509,21 +577,27 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
     // row i of A -> TMEM lane i
     const float4* Ar = reinterpret_cast<const float4*>(A + (size_t)m * kDD + (size_t)i * kD);
 #pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
-      uint32_t v[32];
+    for (int q = 0; q < 4; q += 2) {
+      uint32_t v[32], w[32];
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const float4 x = __ldg(Ar + 8 * q + c);
+        const float4 x = __ldg(Ar + 8 * q + c), y = __ldg(Ar + 8 * q + 8 + c);
         v[4 * c] = __float_as_uint(x.x); v[4 * c + 1] = __float_as_uint(x.y);
         v[4 * c + 2] = __float_as_uint(x.z); v[4 * c + 3] = __float_as_uint(x.w);
+        w[4 * c] = __float_as_uint(y.x); w[4 * c + 1] = __float_as_uint(y.y);
+        w[4 * c + 2] = __float_as_uint(y.z); w[4 * c + 3] = __float_as_uint(y.w);
       }
       tmem_st32(lb + tA + 32u * q, v);
+      tmem_st32(lb + tA + 32u * (q + 1), w);
     }
+    const int mnext = m + gridDim.x * C::GROUPS;
+    if (i == 0 && mnext < FH)   // the group's next matrix: into L2 while this one is swept
+      bulk_prefetch_l2(A + (size_t)mnext * kDD, (uint32_t)(kDD * sizeof(float)));
     tmem_wait_st();
     tc_fence_before();
     named_bar_sync(bid, 128);
     tc_fence_after();
-    if (!sweep_inverse_tmem(tA, tW, lb, swb, bid, sbar, sweep_phase, abort_flag, i, gw, lane)) break;
+    if (!sweep_inverse_tmem(tA, lb, swb, bid, bid + C::GROUPS, sbar, sweep_phase, abort_flag, i, gw, lane, g)) break;
     // M = -(swept matrix): row i -> operand image row i (k index), debug copy
     uint8_t* img = Mimg + (size_t)m * kImgBytes;
 #pragma unroll 1
@@ -804,7 +878,7 @@ struct ReadoutCfg {
   static constexpr uint32_t OFF_G = kImgBytes + 2 * TILE_BYTES; // 2 x 32 KB
   static constexpr uint32_t OFF_W = kImgBytes + 4 * TILE_BYTES; // 128 floats
   static constexpr uint32_t BAR_OFF = OFF_W + 512;
-  // qfull[2], qempty[2], gfull[2], gempty[2], tfull[2], tempty[2], sready, drain
+  // qfull[2], qempty[2], gfull[2], gout[2], tfull[2], tempty[2], sready, drain
   static constexpr int NBAR = 14;
   static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
 };
@@ -831,6 +905,7 @@ __device__ __forceinline__ void tile_coords(const ReadoutGeom& g, long long gt, 
 
 __global__ void __launch_bounds__(ReadoutCfg::THREADS, 1)
 k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
+             const __grid_constant__ CUtensorMap tmO,
              const float* __restrict__ w, const float* __restrict__ states,
              __nv_bfloat16* __restrict__ out, ReadoutGeom g, float eps) {
   using C = ReadoutCfg;
@@ -838,7 +913,7 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
   auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
-  const int QFULL = 0, QEMPTY = 2, GFULL = 4, GEMPTY = 6, TFULL = 8, TEMPTY = 10, SREADY = 12, DRAIN = 13;
+  const int QFULL = 0, QEMPTY = 2, GFULL = 4, GOUT = 6, TFULL = 8, TEMPTY = 10, SREADY = 12, DRAIN = 13;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sw = reinterpret_cast<float*>(smem + C::OFF_W);
@@ -853,7 +928,7 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       mbar_init(BAR(QFULL + s), 1);
       mbar_init(BAR(QEMPTY + s), 1);
       mbar_init(BAR(GFULL + s), 1);
-      mbar_init(BAR(GEMPTY + s), 128);
+      mbar_init(BAR(GOUT + s), 128);
       mbar_init(BAR(TFULL + s), 1);
       mbar_init(BAR(TEMPTY + s), 128);
     }
@@ -875,26 +950,55 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
   int last_q[2] = {-1, -1}, last_g[2] = {-1, -1};   // producer: last tile issued per stage
 
   if (warp == 4 || warp == 6) {
-    // ---------------- TMA producers: Q tiles (warp 4), gate tiles (warp 6)
+    // ---------------- TMA producers: Q tiles (warp 4); gate tiles (warp 6),
+    // which also sends each output tile out of the gate stage it replaced
     if (lane == 0) {
       const bool is_q = warp == 4;
-      const int FULLB = is_q ? QFULL : GFULL, EMPTYB = is_q ? QEMPTY : GEMPTY;
       const CUtensorMap* map = is_q ? &tmQ : &tmG;
       const uint32_t base = sbase + (is_q ? C::OFF_Q : C::OFF_G);
       int* last = is_q ? last_q : last_g;
+      // output tile of tile index gt (stage s) -> global, when it is a full tile
+      auto store_out = [&](long long gt, uint32_t s) {
+        int bh, c, tr, rows;
+        tile_coords(g, gt, bh, c, tr, rows);
+        if (tr + C::TILE <= rows) {
+          const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.chunk * g.U + tr);
+          const uint32_t src = base + s * C::TILE_BYTES;
+          tma_store_2d(&tmO, src, 0, row0);
+          tma_store_2d(&tmO, src + C::TILE_BYTES / 2, 64, row0);
+          bulk_commit_group();
+        }
+      };
+      bool ok = true;
       int k = 0;
       for (long long gt = t_begin; gt < t_end; ++gt, ++k) {
         int bh, c, tr, rows;
         tile_coords(g, gt, bh, c, tr, rows);
         const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.chunk * g.U + tr);
         const uint32_t s = (uint32_t)k & 1u, ph = ((uint32_t)k >> 1) & 1u;
-        if (!mbar_wait(BAR(EMPTYB + s), ph ^ 1u, abort_flag)) break;
+        if (is_q) {
+          if (!mbar_wait(BAR(QEMPTY + s), ph ^ 1u, abort_flag)) { ok = false; break; }
+        } else if (k >= 2) {   // the stage holds tile k-2's output: send it, let the copy read it
+          if (!mbar_wait(BAR(GOUT + s), ph ^ 1u, abort_flag)) { ok = false; break; }
+          store_out(gt - 2, s);
+          bulk_wait_read_all();
+        }
+        const int FULLB = is_q ? QFULL : GFULL;
         mbar_arrive_expect_tx(BAR(FULLB + s), C::TILE_BYTES);
         const uint32_t dst = base + s * C::TILE_BYTES;
         tma_load_2d(dst, map, 0, row0, BAR(FULLB + s));
         tma_load_2d(dst + C::TILE_BYTES / 2, map, 64, row0, BAR(FULLB + s));
         last[s] = k;
       }
+      if (!is_q && ok) {   // the last two output tiles
+        const int n = k;
+        for (int kk = max(0, n - 2); kk < n; ++kk) {
+          const uint32_t s = (uint32_t)kk & 1u, ph = ((uint32_t)kk >> 1) & 1u;
+          if (!mbar_wait(BAR(GOUT + s), ph, abort_flag)) break;
+          store_out(t_begin + kk, s);
+        }
+      }
+      if (!is_q) bulk_wait_all();   // output copies complete before the CTA retires
     }
   } else if (warp == 5) {
     // ---------------- MMA issuer
@@ -1003,6 +1107,9 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(GFULL + s), ph, abort_flag))) break;
       const uint32_t gt_s = sbase + C::OFF_G + s * C::TILE_BYTES;
       const bool valid = tr + r < rows;
+      // a tile inside its chunk leaves by TMA from the gate stage (y replaces
+      // g in place); the chunk's last, partial tile by per-row stores
+      const bool tma_out = tr + C::TILE <= rows;
       __nv_bfloat16* orow = out + ((size_t)bh * tokens_per_head + (size_t)c * g.chunk * g.U + tr + r) * kD;
 #pragma unroll
       for (int cc = 0; cc < 16; ++cc) {
@@ -1023,9 +1130,11 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
           const float y1 = fmaf(a1, tanh_approx(0.5f * g1), a1);
           yw[q] = pack_bf16(y0, y1);
         }
-        if (valid) *reinterpret_cast<uint4*>(orow + cc * 8) = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+        if (tma_out) st_shared_v4(gt_s + off, make_uint4(yw[0], yw[1], yw[2], yw[3]));
+        else if (valid) *reinterpret_cast<uint4*>(orow + cc * 8) = make_uint4(yw[0], yw[1], yw[2], yw[3]);
       }
-      mbar_arrive(BAR(GEMPTY + s));
+      if (tma_out) fence_proxy_async_smem();
+      mbar_arrive(BAR(GOUT + s));
     }
   }
 
@@ -1178,15 +1287,16 @@ inline int launch_readout(const void* Q, const void* G, const float* w, const fl
   g.tph = (NC - 1) * g.tpc + g.tlast;
   g.total = (long long)BH * g.tph;
   const uint64_t rows = (uint64_t)BH * T * U;
-  CUtensorMap tmQ, tmG;
-  if (!encode_bf16_2d(&tmQ, Q, rows, ReadoutCfg::TILE) || !encode_bf16_2d(&tmG, G, rows, ReadoutCfg::TILE))
+  CUtensorMap tmQ, tmG, tmO;
+  if (!encode_bf16_2d(&tmQ, Q, rows, ReadoutCfg::TILE) || !encode_bf16_2d(&tmG, G, rows, ReadoutCfg::TILE) ||
+      !encode_bf16_2d(&tmO, out, rows, ReadoutCfg::TILE))
     return VDA_ERR_CUDA;
   if (cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ReadoutCfg::SMEM) !=
       cudaSuccess)
     return VDA_ERR_CUDA;
   const int grid = (int)std::min<long long>(g.total, (long long)num_sms());
   k_readout_tc<<<grid, ReadoutCfg::THREADS, ReadoutCfg::SMEM, s>>>(
-      tmQ, tmG, w, states, static_cast<__nv_bfloat16*>(out), g, eps);
+      tmQ, tmG, tmO, w, states, static_cast<__nv_bfloat16*>(out), g, eps);
   return launch_status("k_readout_tc");
 }
 
