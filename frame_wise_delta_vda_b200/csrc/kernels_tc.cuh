@@ -47,7 +47,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 //
 // Persistent CTAs (one per SM) walk frame-heads fh = blockIdx.x + i*grid.
 // Warps: 0-3 epilogue (TMEM -> A and B, fp32, standard layouts, coalesced),
-//        4-7 scale (beta*K hi/lo), 8 TMA producer, 9 MMA issuer + TMEM
+//        4-11 scale (beta*K hi/lo), 12 TMA producer, 13 MMA issuer + TMEM
 //        owner.  Two TMEM accumulators: the epilogue of one frame-head
 //        overlaps the MMAs of the next.
 // Stage s holds K0 K1 V0 V1 (TMA), H0 H1 (hi), L0 L1 (lo): 8 x 8 KB.
@@ -62,7 +62,10 @@ struct StatsCfg {
   static constexpr uint32_t OFF_H = 4 * BLK;
   static constexpr uint32_t OFF_L = 6 * BLK;
   static constexpr uint32_t STAGE = 8 * BLK;         // 65536
-  static constexpr int THREADS = 320;
+  static constexpr int NSCALE = 256;                 // scale threads: 64 rows x 4 column quarters
+  static constexpr int WARP_PROD = 4 + NSCALE / 32;  // TMA producer
+  static constexpr int WARP_MMA = WARP_PROD + 1;     // MMA issuer + TMEM owner
+  static constexpr int THREADS = 32 * (WARP_MMA + 1);
   static constexpr uint32_t BAR_OFF = NST * STAGE;
   static constexpr int NBAR = 3 * NST + 5;
   static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
@@ -130,7 +133,7 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
   if (tid == 0) {
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(BAR(FULL + s), 1);
-      mbar_init(BAR(SCALED + s), 128);
+      mbar_init(BAR(SCALED + s), C::NSCALE);
       mbar_init(BAR(EMPTY + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -141,7 +144,7 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == C::WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -153,7 +156,7 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
   int last_it[C::NST];   // producer: last iteration issued on each stage
   for (int s = 0; s < C::NST; ++s) last_it[s] = -1;
 
-  if (warp == 8) {
+  if (warp == C::WARP_PROD) {
     // ---------------- TMA producer
     if (lane == 0) {
       uint32_t it = 0;
@@ -172,7 +175,7 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == C::WARP_MMA) {
     // ---------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdN256 = idesc_bf16(128, 256, 1, 1);
@@ -207,9 +210,10 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ---------------- beta * K, split into bf16 hi + lo (same swizzled position)
+    // ---------------- beta * K, split into bf16 hi + lo (same swizzled position):
+    // thread = (row r, quarter qt) of the 64 x 128 tile; 4 chunks of 8 channels
     const int st_id = tid - 128;
-    const int r = st_id & 63, hb = st_id >> 6;
+    const int r = st_id & 63, qt = st_id >> 6, hb = qt >> 1;
     auto beta_at = [&](int f, int tl) -> float {
       const int u = tl * C::UT + r;
       return (f < FH && u < U) ? __ldg(beta + (size_t)f * U + u) : 0.f;
@@ -226,24 +230,29 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
       if (!mbar_wait(BAR(FULL + s), ph, abort_flag)) break;
       const uint32_t rowb = sbase + s * C::STAGE + hb * C::BLK + (uint32_t)r * 128u;
       const uint32_t ksrc = rowb + C::OFF_KV, hdst = rowb + C::OFF_H, ldst = rowb + C::OFF_L;
+      // the loads first: the shared-memory accesses are ordered asm statements,
+      // so this order is what lets the arithmetic overlap them
+      uint32_t pos[4];
+      uint4 kvs[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t p = (uint32_t)((c + r) & 7) * 16u;   // rotate chunks across rows: conflict-free
-        const uint4 kv = ld_shared_v4(ksrc + p);
-        const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+      for (int c = 0; c < 4; ++c) {
+        pos[c] = (uint32_t)((4 * (qt & 1) + c + r) & 7) * 16u;   // rotated across rows: conflict-free
+        kvs[c] = ld_shared_v4(ksrc + pos[c]);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t w[4] = {kvs[c].x, kvs[c].y, kvs[c].z, kvs[c].w};
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float x0 = __uint_as_float(w[q] << 16) * b;
           const float x1 = __uint_as_float(w[q] & 0xFFFF0000u) * b;
-          float h0, l0, h1, l1;
-          split_bf16(x0, h0, l0);
-          split_bf16(x1, h1, l1);
-          hw[q] = pack_bf16(h0, h1);
-          lw[q] = pack_bf16(l0, l1);
+          hw[q] = pack_bf16(x0, x1);   // hi = rn(x)
+          const float h0 = __uint_as_float(hw[q] << 16), h1 = __uint_as_float(hw[q] & 0xFFFF0000u);
+          lw[q] = pack_bf16(x0 - h0, x1 - h1);   // lo = rn(x - hi)
         }
-        st_shared_v4(hdst + p, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-        st_shared_v4(ldst + p, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+        st_shared_v4(hdst + pos[c], make_uint4(hw[0], hw[1], hw[2], hw[3]));
+        st_shared_v4(ldst + pos[c], make_uint4(lw[0], lw[1], lw[2], lw[3]));
       }
       fence_proxy_async_smem();
       mbar_arrive(BAR(SCALED + s));
@@ -265,32 +274,28 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
       float* Af = A_out + (size_t)fh * kDD;
       float* Bf = B_out + (size_t)fh * kDD;
 #pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        uint32_t v0[32], v1[32];
-        tmem_ld32(lb + tA + 64u * q, v0);
-        tmem_ld32(lb + tA + 64u * q + 32u, v1);
+      for (int q = 0; q < 8; ++q) {
+        uint32_t v0[32];
+        tmem_ld32(lb + tA + 32u * q, v0);
         tmem_wait_ld();
-        if (q == 3) {
+        if (q == 7) {
           tc_fence_before();
           mbar_arrive(BAR(TEMPTY + buf));
         }
-        float* dst = q < 2 ? Af + (size_t)(64 * q) * kD : Bf + (size_t)(64 * (q - 2)) * kD;
+        float* dst = q < 4 ? Af + (size_t)(32 * q) * kD : Bf + (size_t)(32 * (q - 4)) * kD;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          dst[(size_t)c * kD + i] = __uint_as_float(v0[c]);
-          dst[(size_t)(c + 32) * kD + i] = __uint_as_float(v1[c]);
-        }
+        for (int c = 0; c < 32; ++c) dst[(size_t)c * kD + i] = __uint_as_float(v0[c]);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == C::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (warp == 8 && lane == 0 && *abort_flag) {  // let issued copies land before the CTA exits
+  if (warp == C::WARP_PROD && lane == 0 && *abort_flag) {  // let issued copies land before the CTA exits
     for (int s = 0; s < C::NST; ++s)
       if (last_it[s] >= 0) mbar_wait_drain(BAR(FULL + s), ((uint32_t)last_it[s] / C::NST) & 1u);
   }
