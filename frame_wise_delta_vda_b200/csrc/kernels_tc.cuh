@@ -865,26 +865,32 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
 // with Q from TMA (K-major, 128-B swizzle) and the S~ image in shared memory,
 // built by the epilogue warps whenever the run enters a new (b, h, chunk):
 //   S~ = fwd[max(0, c - w)] + rev[min(NC, c + w + 1)]   (Appendix A.3)
-// TMEM lane = token row: RMSNorm is a per-thread sum of squares.  Gates come
-// through TMA as well; outputs are stored as 16-B vectors, rows past the
-// chunk end are skipped.  The gate is sigmoid(g) = (1 + tanh(g/2)) / 2 with
-// the hardware tanh (one XU instruction per element), and the factor 1/2 is
-// folded into the RMSNorm weight held in shared memory.
-// Warps 0-3: epilogue + S~ builder; warp 4: Q producer; warp 5: MMA issuer;
-// warp 6: gate producer (separate producers keep Q loads running ahead of
+// TMEM lane = token row: two epilogue warps share a row quarter (the warps
+// e and e + 4 reach the same TMEM lanes), each sums the squares of the whole
+// row, in the same order, and writes one 64-column half.  Gates come through
+// TMA as well; each output replaces its gate in the gate stage, and the gate
+// producer sends the tile out by TMA (the partial tile at a chunk end is
+// stored row by row instead).  The gate is sigmoid(g) = (1 + tanh(g/2)) / 2
+// with the hardware tanh (one XU instruction per element), and the factor
+// 1/2 is folded into the RMSNorm weight held in shared memory.
+// Warps 0-7: epilogue + S~ builder; warp 8: Q producer; warp 9: MMA issuer;
+// warp 10: gate producer (separate producers keep Q loads running ahead of
 // the epilogue's release of gate stages).
 // ===========================================================================
 struct ReadoutCfg {
-  static constexpr int THREADS = 224;
+  static constexpr int NEPI = 256;                             // epilogue threads (warps 0-7)
+  static constexpr int WARP_Q = 8, WARP_MMA = 9, WARP_G = 10;
+  static constexpr int THREADS = 352;
   static constexpr int TILE = 128;
   static constexpr uint32_t TILE_BYTES = TILE * 256;           // 128 rows x 128 bf16
   static constexpr uint32_t OFF_S = 0;                         // S~ hi (32 KB) + lo (32 KB)
   static constexpr uint32_t OFF_Q = kImgBytes;                 // 2 x 32 KB
-  static constexpr uint32_t OFF_G = kImgBytes + 2 * TILE_BYTES; // 2 x 32 KB
-  static constexpr uint32_t OFF_W = kImgBytes + 4 * TILE_BYTES; // 128 floats
+  static constexpr int NG = 2;                                  // gate stages (also hold the output)
+  static constexpr uint32_t OFF_G = kImgBytes + 2 * TILE_BYTES; // NG x 32 KB
+  static constexpr uint32_t OFF_W = OFF_G + NG * TILE_BYTES;    // 128 floats
   static constexpr uint32_t BAR_OFF = OFF_W + 512;
-  // qfull[2], qempty[2], gfull[2], gout[2], tfull[2], tempty[2], sready, drain
-  static constexpr int NBAR = 14;
+  // qfull[2], qempty[2], gfull[NG], gout[NG], tfull[2], tempty[2], sready, drain
+  static constexpr int NBAR = 10 + 2 * NG;
   static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
 };
 
@@ -918,7 +924,8 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
   auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
-  const int QFULL = 0, QEMPTY = 2, GFULL = 4, GOUT = 6, TFULL = 8, TEMPTY = 10, SREADY = 12, DRAIN = 13;
+  const int QFULL = 0, QEMPTY = 2, GFULL = 4, GOUT = 4 + C::NG, TFULL = 4 + 2 * C::NG, TEMPTY = TFULL + 2,
+            SREADY = TFULL + 4, DRAIN = TFULL + 5;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sw = reinterpret_cast<float*>(smem + C::OFF_W);
@@ -932,18 +939,20 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(QFULL + s), 1);
       mbar_init(BAR(QEMPTY + s), 1);
-      mbar_init(BAR(GFULL + s), 1);
-      mbar_init(BAR(GOUT + s), 128);
       mbar_init(BAR(TFULL + s), 1);
-      mbar_init(BAR(TEMPTY + s), 128);
+      mbar_init(BAR(TEMPTY + s), C::NEPI);
     }
-    mbar_init(BAR(SREADY), 128);
+    for (int s = 0; s < C::NG; ++s) {
+      mbar_init(BAR(GFULL + s), 1);
+      mbar_init(BAR(GOUT + s), C::NEPI);
+    }
+    mbar_init(BAR(SREADY), C::NEPI);
     mbar_init(BAR(DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (tid < kD) sw[tid] = 0.5f * w[tid];
-  if (warp == 5) {
+  if (warp == C::WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), 256);
     tmem_relinquish();
   }
@@ -952,16 +961,18 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const long long tokens_per_head = (long long)g.T * g.U;
-  int last_q[2] = {-1, -1}, last_g[2] = {-1, -1};   // producer: last tile issued per stage
+  int last_q[2] = {-1, -1}, last_g[C::NG];   // producer: last tile issued per stage
+  for (int q = 0; q < C::NG; ++q) last_g[q] = -1;
 
-  if (warp == 4 || warp == 6) {
-    // ---------------- TMA producers: Q tiles (warp 4); gate tiles (warp 6),
+  if (warp == C::WARP_Q || warp == C::WARP_G) {
+    // ---------------- TMA producers: Q tiles; gate tiles,
     // which also sends each output tile out of the gate stage it replaced
     if (lane == 0) {
-      const bool is_q = warp == 4;
+      const bool is_q = warp == C::WARP_Q;
       const CUtensorMap* map = is_q ? &tmQ : &tmG;
       const uint32_t base = sbase + (is_q ? C::OFF_Q : C::OFF_G);
       int* last = is_q ? last_q : last_g;
+      const int ns = is_q ? 2 : C::NG;
       // output tile of tile index gt (stage s) -> global, when it is a full tile
       auto store_out = [&](long long gt, uint32_t s) {
         int bh, c, tr, rows;
@@ -980,12 +991,12 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         int bh, c, tr, rows;
         tile_coords(g, gt, bh, c, tr, rows);
         const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.chunk * g.U + tr);
-        const uint32_t s = (uint32_t)k & 1u, ph = ((uint32_t)k >> 1) & 1u;
+        const uint32_t s = (uint32_t)(k % ns), ph = (uint32_t)(k / ns) & 1u;
         if (is_q) {
           if (!mbar_wait(BAR(QEMPTY + s), ph ^ 1u, abort_flag)) { ok = false; break; }
-        } else if (k >= 2) {   // the stage holds tile k-2's output: send it, let the copy read it
+        } else if (k >= C::NG) {   // the stage holds tile k-NG's output: send it, let the copy read it
           if (!mbar_wait(BAR(GOUT + s), ph ^ 1u, abort_flag)) { ok = false; break; }
-          store_out(gt - 2, s);
+          store_out(gt - C::NG, s);
           bulk_wait_read_all();
         }
         const int FULLB = is_q ? QFULL : GFULL;
@@ -995,17 +1006,17 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         tma_load_2d(dst + C::TILE_BYTES / 2, map, 64, row0, BAR(FULLB + s));
         last[s] = k;
       }
-      if (!is_q && ok) {   // the last two output tiles
+      if (!is_q && ok) {   // the last NG output tiles
         const int n = k;
-        for (int kk = max(0, n - 2); kk < n; ++kk) {
-          const uint32_t s = (uint32_t)kk & 1u, ph = ((uint32_t)kk >> 1) & 1u;
+        for (int kk = max(0, n - C::NG); kk < n; ++kk) {
+          const uint32_t s = (uint32_t)(kk % C::NG), ph = (uint32_t)(kk / C::NG) & 1u;
           if (!mbar_wait(BAR(GOUT + s), ph, abort_flag)) break;
           store_out(t_begin + kk, s);
         }
       }
       if (!is_q) bulk_wait_all();   // output copies complete before the CTA retires
     }
-  } else if (warp == 5) {
+  } else if (warp == C::WARP_MMA) {
     // ---------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t kId = idesc_bf16(128, 128, 0, 0);   // both K-major
@@ -1041,24 +1052,25 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (thread r = token row r of the tile) + S~ builder
-    const int r = warp * 32 + lane;
-    const uint32_t trow_base = tmem + ((uint32_t)(warp * 32) << 16);
+    // ---------------- epilogue + S~ builder: thread = (token row r, column half ch)
+    const int r = (warp & 3) * 32 + lane, ch = warp >> 2;
+    const uint32_t trow_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t simg_s = sbase + C::OFF_S;
-    const uint32_t sw_s = sbase + C::OFF_W;
+    const uint32_t sw_s = sbase + C::OFF_W + 256u * (uint32_t)ch;   // w/2 of this half
     int k = 0, prev_bh = -1, prev_c = -1;
     const size_t sdir = (size_t)g.BH * (size_t)(g.NC + 1) * kDD;
     for (long long gt = t_begin; gt < t_end; ++gt, ++k) {
       int bh, c, tr, rows;
       tile_coords(g, gt, bh, c, tr, rows);
       if (bh != prev_bh || c != prev_c) {
-        // build S~ = fwd[max(0, c-w)] + rev[min(NC, c+w+1)]: thread r writes row i = r
+        // build S~ = fwd[max(0, c-w)] + rev[min(NC, c+w+1)]: row i = r, this half's columns
         const int jf = max(0, c - g.window), jr = min(g.NC, c + g.window + 1);
-        const float* Sf = states + (size_t)bh * (size_t)(g.NC + 1) * kDD + (size_t)jf * kDD + (size_t)r * kD;
+        const float* Sf =
+            states + (size_t)bh * (size_t)(g.NC + 1) * kDD + (size_t)jf * kDD + (size_t)r * kD + 64 * ch;
         const float* Sr = states + sdir + (size_t)bh * (size_t)(g.NC + 1) * kDD + (size_t)jr * kD * kD +
-                          (size_t)r * kD;
+                          (size_t)r * kD + 64 * ch;
 #pragma unroll 4
-        for (int cc = 0; cc < 16; ++cc) {
+        for (int cc = 0; cc < 8; ++cc) {
           const float4 f0 = __ldg(reinterpret_cast<const float4*>(Sf + cc * 8));
           const float4 f1 = __ldg(reinterpret_cast<const float4*>(Sf + cc * 8 + 4));
           const float4 r0v = __ldg(reinterpret_cast<const float4*>(Sr + cc * 8));
@@ -1074,7 +1086,7 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             hw[q] = pack_bf16(h0, h1);
             lw[q] = pack_bf16(l0, l1);
           }
-          const uint32_t off = ximg_offset(r, cc * 8);   // row i = r, columns k = 8cc..8cc+7
+          const uint32_t off = ximg_offset(r, 64 * ch + cc * 8);   // row i = r, columns k
           st_shared_v4(simg_s + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
           st_shared_v4(simg_s + kImgHalf + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
         }
@@ -1086,74 +1098,97 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       const uint32_t s = (uint32_t)k & 1u, ph = ((uint32_t)k >> 1) & 1u;
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(TFULL + s), ph, abort_flag))) break;
       tc_fence_after();
-      float o[kD];
+      // sum of squares over the whole row (both halves, fixed order); keep this half
+      float o[64];
+      float ss = 0.f;
       const uint32_t trow = trow_base + s * 128u;
-      {
-        uint32_t v0[32], v1[32], v2[32], v3[32];
-        tmem_ld32(trow, v0);
-        tmem_ld32(trow + 32, v1);
-        tmem_ld32(trow + 64, v2);
-        tmem_ld32(trow + 96, v3);
+#pragma unroll
+      for (int j2 = 0; j2 < 2; ++j2) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(trow + 64u * j2, v0);
+        tmem_ld32(trow + 64u * j2 + 32u, v1);
         tmem_wait_ld();
 #pragma unroll
         for (int c2 = 0; c2 < 32; ++c2) {
-          o[c2] = __uint_as_float(v0[c2]);
-          o[32 + c2] = __uint_as_float(v1[c2]);
-          o[64 + c2] = __uint_as_float(v2[c2]);
-          o[96 + c2] = __uint_as_float(v3[c2]);
+          const float a0 = __uint_as_float(v0[c2]);
+          ss = fmaf(a0, a0, ss);
+        }
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) {
+          const float a1 = __uint_as_float(v1[c2]);
+          ss = fmaf(a1, a1, ss);
+        }
+        if (j2 == ch) {
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            o[c2] = __uint_as_float(v0[c2]);
+            o[32 + c2] = __uint_as_float(v1[c2]);
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(BAR(TEMPTY + s));
-      float ss = 0.f;
-#pragma unroll
-      for (int i = 0; i < kD; ++i) ss = fmaf(o[i], o[i], ss);
       const float rinv = rsqrtf(ss * (1.0f / kD) + eps);
-      if (!__all_sync(0xffffffffu, mbar_wait(BAR(GFULL + s), ph, abort_flag))) break;
-      const uint32_t gt_s = sbase + C::OFF_G + s * C::TILE_BYTES;
+      const uint32_t sg = (uint32_t)(k % C::NG), phg = (uint32_t)(k / C::NG) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(GFULL + sg), phg, abort_flag))) break;
+      const uint32_t gt_s = sbase + C::OFF_G + sg * C::TILE_BYTES + (uint32_t)ch * (C::TILE_BYTES / 2);
       const bool valid = tr + r < rows;
       // a tile inside its chunk leaves by TMA from the gate stage (y replaces
       // g in place); the chunk's last, partial tile by per-row stores
       const bool tma_out = tr + C::TILE <= rows;
-      __nv_bfloat16* orow = out + ((size_t)bh * tokens_per_head + (size_t)c * g.chunk * g.U + tr + r) * kD;
+      __nv_bfloat16* orow =
+          out + ((size_t)bh * tokens_per_head + (size_t)c * g.chunk * g.U + tr + r) * kD + 64 * ch;
 #pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        const uint32_t off = (uint32_t)(cc >> 3) * (C::TILE_BYTES / 2) + sw128_offset((uint32_t)r, (uint32_t)((cc & 7) * 8));
-        const uint4 gv = ld_shared_v4(gt_s + off);
-        const float4 wa = ld_shared_f4(sw_s + (uint32_t)cc * 32u);
-        const float4 wb = ld_shared_f4(sw_s + (uint32_t)cc * 32u + 16u);
-        const float wh[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-        uint32_t yw[4];
+      for (int cb = 0; cb < 2; ++cb) {   // 4 chunks of 8 columns at a time, loads first
+        uint4 gv[4];
+        float4 wv[8];
+        uint32_t off[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int i0 = cc * 8 + 2 * q;
-          const float g0 = __uint_as_float(gw[q] << 16), g1 = __uint_as_float(gw[q] & 0xFFFF0000u);
-          // y = w * o * rinv * sigmoid(g),  sigmoid(g) = (1 + tanh(g / 2)) / 2, w/2 in wh
-          const float a0 = o[i0] * rinv * wh[2 * q], a1 = o[i0 + 1] * rinv * wh[2 * q + 1];
-          const float y0 = fmaf(a0, tanh_approx(0.5f * g0), a0);
-          const float y1 = fmaf(a1, tanh_approx(0.5f * g1), a1);
-          yw[q] = pack_bf16(y0, y1);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int cc = 4 * cb + q4;
+          off[q4] = sw128_offset((uint32_t)r, (uint32_t)(cc * 8));
+          gv[q4] = ld_shared_v4(gt_s + off[q4]);
+          wv[2 * q4] = ld_shared_f4(sw_s + (uint32_t)cc * 32u);
+          wv[2 * q4 + 1] = ld_shared_f4(sw_s + (uint32_t)cc * 32u + 16u);
         }
-        if (tma_out) st_shared_v4(gt_s + off, make_uint4(yw[0], yw[1], yw[2], yw[3]));
-        else if (valid) *reinterpret_cast<uint4*>(orow + cc * 8) = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int cc = 4 * cb + q4;
+          const float wh[8] = {wv[2 * q4].x, wv[2 * q4].y, wv[2 * q4].z, wv[2 * q4].w,
+                               wv[2 * q4 + 1].x, wv[2 * q4 + 1].y, wv[2 * q4 + 1].z, wv[2 * q4 + 1].w};
+          const uint32_t gw[4] = {gv[q4].x, gv[q4].y, gv[q4].z, gv[q4].w};
+          uint32_t yw[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int i0 = cc * 8 + 2 * q;
+            const float g0 = __uint_as_float(gw[q] << 16), g1 = __uint_as_float(gw[q] & 0xFFFF0000u);
+            // y = w * o * rinv * sigmoid(g),  sigmoid(g) = (1 + tanh(g / 2)) / 2, w/2 in wh
+            const float a0 = o[i0] * rinv * wh[2 * q], a1 = o[i0 + 1] * rinv * wh[2 * q + 1];
+            const float y0 = fmaf(a0, tanh_approx(0.5f * g0), a0);
+            const float y1 = fmaf(a1, tanh_approx(0.5f * g1), a1);
+            yw[q] = pack_bf16(y0, y1);
+          }
+          if (tma_out) st_shared_v4(gt_s + off[q4], make_uint4(yw[0], yw[1], yw[2], yw[3]));
+          else if (valid) *reinterpret_cast<uint4*>(orow + cc * 8) = make_uint4(yw[0], yw[1], yw[2], yw[3]);
+        }
       }
       if (tma_out) fence_proxy_async_smem();
-      mbar_arrive(BAR(GOUT + s));
+      mbar_arrive(BAR(GOUT + sg));
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == C::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
-  if ((warp == 4 || warp == 6) && lane == 0 && *abort_flag) {  // let issued copies land before exit
-    const int* last = warp == 4 ? last_q : last_g;
-    const int FULLB = warp == 4 ? QFULL : GFULL;
-    for (int s = 0; s < 2; ++s)
-      if (last[s] >= 0) mbar_wait_drain(BAR(FULLB + s), ((uint32_t)last[s] >> 1) & 1u);
+  if ((warp == C::WARP_Q || warp == C::WARP_G) && lane == 0 && *abort_flag) {  // let issued copies land
+    const int* last = warp == C::WARP_Q ? last_q : last_g;
+    const int FULLB = warp == C::WARP_Q ? QFULL : GFULL;
+    const int ns = warp == C::WARP_Q ? 2 : C::NG;
+    for (int s = 0; s < ns; ++s)
+      if (last[s] >= 0) mbar_wait_drain(BAR(FULLB + s), (uint32_t)(last[s] / ns) & 1u);
   }
 }
 
