@@ -315,14 +315,14 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
 // products, ~16 significant bits).  The 16 x 16 sweep is the sequential part,
 // so it runs one block ahead: while the tensor cores update the matrix with
 // block P, the warp owning the next block Q brings A_QQ up to date itself
-// (A_QQ + (C G)_Q C_Q^T in fp32) and sweeps it.  Three warpgroups per CTA
-// work on three matrices at once (own TMEM columns, shared-memory workspace,
+// (A_QQ + (C G)_Q C_Q^T in fp32) and sweeps it.  Four warpgroups per CTA
+// work on four matrices at once (own TMEM columns, shared-memory workspace,
 // named barrier and completion barrier).  In: A rows (fp32, from
 // k_stats_tc).  Out: the scan's M operand image (element (j, k) = M[k][j],
 // MN-major, 128-B swizzle, bf16 hi / lo halves) and optionally M in fp32.
 // ===========================================================================
 struct InvCfg {
-  static constexpr int GROUPS = 3;
+  static constexpr int GROUPS = 4;
   static constexpr int THREADS = 128 * GROUPS;
   static constexpr uint32_t TCOLS = 128;     // TMEM columns per group: the matrix
   static constexpr uint32_t SW_BYTES = 28672; // per-group workspace (see SW_* below)
