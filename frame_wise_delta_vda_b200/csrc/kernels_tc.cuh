@@ -50,24 +50,27 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 //        4-11 scale (beta*K hi/lo), 12 TMA producer, 13 MMA issuer + TMEM
 //        owner.  Two TMEM accumulators: the epilogue of one frame-head
 //        overlaps the MMAs of the next.
-// Stage s holds K0 K1 V0 V1 (TMA), H0 H1 (hi), L0 L1 (lo): 8 x 8 KB.
+// Load stage s holds K0 K1 V0 V1 (TMA, 4 x 8 KB; four stages keep 128 KB of
+// loads in flight); scaled buffer b holds H0 H1 (hi), L0 L1 (lo) (4 x 8 KB,
+// two buffers: they live only from the scaling to the MMAs).
 // TMEM: two 256-column accumulators (512 columns), so the epilogue of one
 // frame-head overlaps the MMAs of the next.
 // ===========================================================================
 struct StatsCfg {
   static constexpr int UT = 64;
-  static constexpr int NST = 3;
+  static constexpr int NST = 4;                      // load stages
+  static constexpr int NSC = 2;                      // scaled buffers
   static constexpr uint32_t BLK = UT * 128;          // 8192
-  static constexpr uint32_t OFF_KV = 0;
-  static constexpr uint32_t OFF_H = 4 * BLK;
-  static constexpr uint32_t OFF_L = 6 * BLK;
-  static constexpr uint32_t STAGE = 8 * BLK;         // 65536
+  static constexpr uint32_t STAGE = 4 * BLK;         // K0 K1 V0 V1
+  static constexpr uint32_t SCBUF = 4 * BLK;         // H0 H1 L0 L1
+  static constexpr uint32_t OFF_SC = NST * STAGE;
+  static constexpr uint32_t OFF_L = 2 * BLK;         // lo half within a scaled buffer
   static constexpr int NSCALE = 256;                 // scale threads: 64 rows x 4 column quarters
   static constexpr int WARP_PROD = 4 + NSCALE / 32;  // TMA producer
   static constexpr int WARP_MMA = WARP_PROD + 1;     // MMA issuer + TMEM owner
   static constexpr int THREADS = 32 * (WARP_MMA + 1);
-  static constexpr uint32_t BAR_OFF = NST * STAGE;
-  static constexpr int NBAR = 3 * NST + 5;
+  static constexpr uint32_t BAR_OFF = OFF_SC + NSC * SCBUF;
+  static constexpr int NBAR = 2 * NST + 2 * NSC + 5;
   static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
 };
 
@@ -124,8 +127,8 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
   const uint32_t sbase = smem_u32(smem);
   auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
   // barrier indices
-  const int FULL = 0, SCALED = C::NST, EMPTY = 2 * C::NST, TFULL = 3 * C::NST, TEMPTY = 3 * C::NST + 2,
-            DRAIN = 3 * C::NST + 4;
+  const int FULL = 0, EMPTY = C::NST, SCALED = 2 * C::NST, SEMPTY = 2 * C::NST + C::NSC,
+            TFULL = 2 * C::NST + 2 * C::NSC, TEMPTY = TFULL + 2, DRAIN = TFULL + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -133,8 +136,11 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
   if (tid == 0) {
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(BAR(FULL + s), 1);
-      mbar_init(BAR(SCALED + s), C::NSCALE);
       mbar_init(BAR(EMPTY + s), 1);
+    }
+    for (int b = 0; b < C::NSC; ++b) {
+      mbar_init(BAR(SCALED + b), C::NSCALE);
+      mbar_init(BAR(SEMPTY + b), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(BAR(TFULL + b), 1);
@@ -187,19 +193,23 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
         tc_fence_after();
         const uint32_t d = tmem + buf * 256u;
         for (int tile = 0; tile < nt; ++tile, ++it) {
-          const uint32_t s = it % C::NST, ph = (it / C::NST) & 1u;
-          if (!mbar_wait(BAR(SCALED + s), ph, abort_flag)) { ok = false; break; }
+          const uint32_t s = it % C::NST;
+          const uint32_t b = it % C::NSC, bph2 = (it / C::NSC) & 1u;
+          // the scale warps waited for the load of stage s before scaling into b
+          if (!mbar_wait(BAR(SCALED + b), bph2, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t st = sbase + s * C::STAGE;
+          const uint32_t sc = sbase + C::OFF_SC + b * C::SCBUF;
 #pragma unroll
           for (int ks = 0; ks < C::UT / 16; ++ks) {
             const uint32_t ko = (uint32_t)ks * 2048u;
-            mma_bf16_ss(d, desc_sw128(st + C::OFF_H + ko, C::BLK, 1024),
-                        desc_sw128(st + C::OFF_KV + ko, C::BLK, 1024), kIdN256, (tile | ks) != 0);
-            mma_bf16_ss(d, desc_sw128(st + C::OFF_L + ko, C::BLK, 1024),
-                        desc_sw128(st + C::OFF_KV + ko, C::BLK, 1024), kIdN256, 1u);
+            mma_bf16_ss(d, desc_sw128(sc + ko, C::BLK, 1024),
+                        desc_sw128(st + ko, C::BLK, 1024), kIdN256, (tile | ks) != 0);
+            mma_bf16_ss(d, desc_sw128(sc + C::OFF_L + ko, C::BLK, 1024),
+                        desc_sw128(st + ko, C::BLK, 1024), kIdN256, 1u);
           }
           mma_commit(BAR(EMPTY + s));
+          mma_commit(BAR(SEMPTY + b));
         }
         if (!ok) break;
         mma_commit(BAR(TFULL + buf));
@@ -227,9 +237,12 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
       if (ntile == nt) { ntile = 0; nfh += gridDim.x; }
       b_next = beta_at(nfh, ntile);
       const uint32_t s = it % C::NST, ph = (it / C::NST) & 1u;
+      const uint32_t sb = it % C::NSC, sph = (it / C::NSC) & 1u;
       if (!mbar_wait(BAR(FULL + s), ph, abort_flag)) break;
-      const uint32_t rowb = sbase + s * C::STAGE + hb * C::BLK + (uint32_t)r * 128u;
-      const uint32_t ksrc = rowb + C::OFF_KV, hdst = rowb + C::OFF_H, ldst = rowb + C::OFF_L;
+      if (!mbar_wait(BAR(SEMPTY + sb), sph ^ 1u, abort_flag)) break;
+      const uint32_t ksrc = sbase + s * C::STAGE + hb * C::BLK + (uint32_t)r * 128u;
+      const uint32_t hdst = sbase + C::OFF_SC + sb * C::SCBUF + hb * C::BLK + (uint32_t)r * 128u;
+      const uint32_t ldst = hdst + C::OFF_L;
       // the loads first: the shared-memory accesses are ordered asm statements,
       // so this order is what lets the arithmetic overlap them
       uint32_t pos[4];
@@ -255,7 +268,7 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
         st_shared_v4(ldst + pos[c], make_uint4(lw[0], lw[1], lw[2], lw[3]));
       }
       fence_proxy_async_smem();
-      mbar_arrive(BAR(SCALED + s));
+      mbar_arrive(BAR(SCALED + sb));
       ++it;
       fh = nfh;
       tile = ntile;
