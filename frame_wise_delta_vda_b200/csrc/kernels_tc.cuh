@@ -665,9 +665,11 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
 // 64h .. 64h+63; lane j holds column j of S.
 // Warps 0-7: state; warps 4h .. 4h+3 own half h (thread j = TMEM lane j of
 // its quarter): read S from TMEM, store boundary states, add B_{t+1}
-// (prefetched into registers), write the X hi/lo image (K-major, 128-B
-// swizzle, one 16 KB image per half and per hi/lo).  The two halves' operand
-// rebuilds run on separate warps, so the tensor pipe sets the step time.
+// (prefetched into registers), write the X hi/lo image.  The image is
+// MN-major (element (k, n) of the MMA's B operand, n contiguous, 128-B
+// swizzle, one 16 KB image per half and per hi/lo): thread j holds k = j for
+// all 64 n of its half, so it writes eight 16-B chunks per hi/lo image.  The
+// two halves' operand rebuilds run on separate warps.
 // Warp 8: bulk-copies the M image of the coming steps (two stages).
 // Warp 9: MMA issuer, TMEM owner.
 // Boundary states: fwd[j] after frames [0, jC), rev[j] after [jC, T).
@@ -679,17 +681,27 @@ struct ScanCfg {
   static constexpr int WARP_MMA = 9;
   static constexpr uint32_t OFF_M = 0;                    // 2 stages x 64 KB
   static constexpr uint32_t OFF_X = 2 * kImgBytes;        // [half][hi/lo] x 16 KB
-  static constexpr uint32_t XIMG = 16384;                 // 64 rows x 128 k bf16
+  static constexpr uint32_t XIMG = 16384;                 // 128 k-rows x 64 n bf16
   static constexpr uint32_t BAR_OFF = 3 * kImgBytes;
   static constexpr int NBAR = 2 + 2 + 2 + 2 + 1;           // mfull[2], mempty[2], xfull[2], dfull[2], drain
   static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
 };
 
-// X image of one 64-row half: element (n, k), n < 64: k-block (k / 64) of
-// 64 rows x 128 B, 128-B swizzle
-__device__ __forceinline__ uint32_t ximg64_offset(int n, int k) {
-  return (uint32_t)(k >> 6) * 8192u + sw128_offset((uint32_t)n, (uint32_t)(k & 63));
+// 8 fp32 values -> one 16-B chunk of the hi image and one of the lo image
+__device__ __forceinline__ void st_chunk_hilo(uint32_t hi_addr, uint32_t lo_addr, const float (&x)[8]) {
+  uint32_t hw[4], lw[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    hw[q] = pack_bf16(x[2 * q], x[2 * q + 1]);   // hi = rn(x)
+    const float h0 = __uint_as_float(hw[q] << 16), h1 = __uint_as_float(hw[q] & 0xFFFF0000u);
+    lw[q] = pack_bf16(x[2 * q] - h0, x[2 * q + 1] - h1);   // lo = rn(x - hi)
+  }
+  st_shared_v4(hi_addr, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+  st_shared_v4(lo_addr, make_uint4(lw[0], lw[1], lw[2], lw[3]));
 }
+
+// element (n, k) of a 128-row K-major operand image: k-block (k / 64) of
+// 128 rows x 128 B, 128-B swizzle
 __device__ __forceinline__ uint32_t ximg_offset(int n, int k) {
   return (uint32_t)(k >> 6) * 16384u + sw128_offset((uint32_t)n, (uint32_t)(k & 63));
 }
@@ -753,7 +765,7 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
   } else if (warp == C::WARP_MMA) {
     // ---------------- MMA issuer: step i = half 0, then half 1
     if (lane == 0) {
-      constexpr uint32_t kId = idesc_bf16(128, 64, 1, 0);   // A (M image) MN-major, B (X half) K-major
+      constexpr uint32_t kId = idesc_bf16(128, 64, 1, 1);   // A (M image) and B (X half) MN-major
       bool ok = true;
       for (int i = 0; ok && i < T; ++i) {
         const uint32_t s = (uint32_t)i & 1u, ph = ((uint32_t)i >> 1) & 1u;
@@ -766,10 +778,9 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
           const uint32_t d = tmem + 64u * (uint32_t)h;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t ao = (uint32_t)ks * 2048u;                                  // 16 k-rows
-            const uint32_t bo = (uint32_t)(ks >> 2) * 8192u + (uint32_t)(ks & 3) * 32u;  // 16 k-columns
-            const uint64_t a_h = desc_sw128(mh + ao, 16384, 1024), a_l = desc_sw128(ml + ao, 16384, 1024);
-            const uint64_t b_h = desc_sw128(xh + bo, 16, 1024), b_l = desc_sw128(xl + bo, 16, 1024);
+            const uint32_t ko = (uint32_t)ks * 2048u;                                  // 16 k-rows
+            const uint64_t a_h = desc_sw128(mh + ko, 16384, 1024), a_l = desc_sw128(ml + ko, 16384, 1024);
+            const uint64_t b_h = desc_sw128(xh + ko, 16384, 1024), b_l = desc_sw128(xl + ko, 16384, 1024);
             mma_bf16_ss(d, a_h, b_h, kId, ks != 0);
             mma_bf16_ss(d, a_h, b_l, kId, 1u);
             mma_bf16_ss(d, a_l, b_h, kId, 1u);
@@ -789,28 +800,27 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
     const float* S0 = dir == 0 ? S0f : S0r;
     float* st = states + ((size_t)dir * BH + bh) * (size_t)(NC + 1) * kDD;
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + 64u * (uint32_t)h;
-    // X image address of element (n2, j) = xs + n2 * 128 + xr[n2 & 7]
-    const uint32_t xs = sbase + C::OFF_X + (uint32_t)h * 2u * C::XIMG + (uint32_t)(j >> 6) * 8192u +
-                        (uint32_t)(j & 7) * 2u;
-    uint32_t xr[8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r) xr[r] = (uint32_t)((((j & 63) >> 3) ^ r) << 4);
+    // X image: row k = j, 16-B chunk c (n2 = 8c .. 8c+7) at ((c ^ (j & 7)) << 4)
+    const uint32_t xrow = sbase + C::OFF_X + (uint32_t)h * 2u * C::XIMG + (uint32_t)j * 128u;
+    const uint32_t jsw = (uint32_t)(j & 7);
     float bnext[64];
 
     // initial state: store it as the first boundary, X_0 = S0 + B_{t0}
     {
       const int j0 = dir == 0 ? 0 : NC;
       const float* B0 = Bm + ((size_t)bh * T + frame_of(0)) * kDD + (size_t)(64 * h) * kD + j;
-#pragma unroll 8
-      for (int n2 = 0; n2 < 64; ++n2) {
-        const int n = 64 * h + n2;
-        const float s0 = S0 ? __ldg(S0 + (size_t)bh * kDD + (size_t)n * kD + j) : 0.f;
-        st[(size_t)j0 * kDD + (size_t)n * kD + j] = s0;
-        float hi, lo;
-        split_bf16(s0 + __ldg(B0 + (size_t)n2 * kD), hi, lo);
-        const uint32_t a = xs + (uint32_t)n2 * 128u + xr[n2 & 7];
-        st_shared_u16(a, bf16_bits(hi));
-        st_shared_u16(a + C::XIMG, bf16_bits(lo));
+#pragma unroll 2
+      for (int c = 0; c < 8; ++c) {
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int n = 64 * h + 8 * c + e;
+          const float s0 = S0 ? __ldg(S0 + (size_t)bh * kDD + (size_t)n * kD + j) : 0.f;
+          st[(size_t)j0 * kDD + (size_t)n * kD + j] = s0;
+          x[e] = s0 + __ldg(B0 + (size_t)(8 * c + e) * kD);
+        }
+        const uint32_t o = xrow + (((uint32_t)c ^ jsw) << 4);
+        st_chunk_hilo(o, o + C::XIMG, x);
       }
       fence_proxy_async_smem();
       mbar_arrive(BAR(XFULL + h));
@@ -836,17 +846,19 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
         uint32_t v[16];
         tmem_ld16(trow + cb * 16, v);
         tmem_wait_ld();
+        if (jb >= 0) {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int n2 = cb * 16 + c;
-          const float sv = __uint_as_float(v[c]);
-          if (jb >= 0) st[(size_t)jb * kDD + (size_t)(64 * h + n2) * kD + j] = sv;
-          if (more) {
-            float hi, lo;
-            split_bf16(sv + bnext[n2], hi, lo);
-            const uint32_t a = xs + (uint32_t)n2 * 128u + xr[c & 7];
-            st_shared_u16(a, bf16_bits(hi));
-            st_shared_u16(a + C::XIMG, bf16_bits(lo));
+          for (int c = 0; c < 16; ++c) st[(size_t)jb * kDD + (size_t)(64 * h + cb * 16 + c) * kD + j] = __uint_as_float(v[c]);
+        }
+        if (more) {
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(v[8 * q + e]) + bnext[cb * 16 + 8 * q + e];
+            const uint32_t c8 = (uint32_t)(2 * cb + q);
+            const uint32_t o = xrow + ((c8 ^ jsw) << 4);
+            st_chunk_hilo(o, o + C::XIMG, x);
           }
         }
       }
