@@ -24,8 +24,9 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-# Stream ids: fixed draw identities (q, k, v, beta, gate, rms weight, text).
-_Q, _K, _V, _BETA, _GATE, _W, _KT, _VT, _BT, _KBASIS = range(10)
+# Stream ids: fixed draw identities (q, k, v, beta, gate, rms weight, text,
+# key basis, decay).
+_Q, _K, _V, _BETA, _GATE, _W, _KT, _VT, _BT, _KBASIS, _ALPHA = range(11)
 
 
 @dataclass(frozen=True)
@@ -44,6 +45,7 @@ class Workload:
     beta_mean: float = 0.0          # beta = sigmoid(N(beta_mean, 1))
     rms_weight: str = "ones"        # "ones" | "jitter" (1 + 0.1 N(0,1))
     text_tokens: int = 0            # > 0: S0 from a text frame
+    alpha_mean: float | None = None  # decay gates alpha = sigmoid(N(alpha_mean, 1)); None: no decay
     notes: str = field(default="", compare=False)
 
     @property
@@ -63,6 +65,13 @@ WORKLOADS = {
                      key_mode="subspace8", beta_mean=2.0),
     "full": Workload("full", 1, 48, 60, 1008, 128, 5, 1, "bf16", 3, text_tokens=256),
     "long": Workload("long", 2, 48, 120, 1008, 128, 5, 1, "bf16", 4, text_tokens=256),
+    # the same shapes with the channel-wise decay gate of Eq. 2 and its bridge
+    "small_decay": Workload("small_decay", 1, 8, 20, 240, 64, 5, 1, "bf16", 11, rms_weight="jitter",
+                            alpha_mean=2.5),
+    "corr_decay": Workload("corr_decay", 1, 16, 30, 1024, 128, 5, 1, "bf16", 12,
+                           key_mode="subspace8", beta_mean=2.0, alpha_mean=2.5),
+    "full_decay": Workload("full_decay", 1, 48, 60, 1008, 128, 5, 1, "bf16", 13, text_tokens=256,
+                           alpha_mean=2.5),
 }
 
 
@@ -108,8 +117,9 @@ def _store(x, dtype):
 
 def head_inputs(wl: Workload, b: int, h: int):
     """Inputs of one (batch, head): dict of q, k, v, gate ([T, U, d], bf16 bits
-    or float32), beta ([T, U] float32) and, if the workload has a text prompt,
-    k_text, v_text ([L, d]) and beta_text ([L] float32)."""
+    or float32), beta ([T, U] float32), alpha ([T, d] float32) if the workload
+    has a decay gate and, if it has a text prompt, k_text, v_text ([L, d]) and
+    beta_text ([L] float32)."""
     T, U, d = wl.T, wl.U, wl.d
     out = {}
     q = _rng(wl.seed, _Q, b, h).standard_normal((T, U, d), dtype=np.float32)
@@ -130,6 +140,10 @@ def head_inputs(wl: Workload, b: int, h: int):
     beta_logit = _rng(wl.seed, _BETA, b, h).standard_normal((T, U), dtype=np.float32) + np.float32(wl.beta_mean)
     out["beta"] = _sigmoid32(beta_logit)
     out["gate"] = _store(_rng(wl.seed, _GATE, b, h).standard_normal((T, U, d), dtype=np.float32), wl.dtype)
+    if wl.alpha_mean is not None:
+        # channel-wise decay gates alpha_t in (0, 1), one per frame and key channel
+        a_logit = _rng(wl.seed, _ALPHA, b, h).standard_normal((T, d), dtype=np.float32) + np.float32(wl.alpha_mean)
+        out["alpha"] = _sigmoid32(a_logit)
     if wl.text_tokens > 0:
         L = wl.text_tokens
         kt = _rng(wl.seed, _KT, b, h).standard_normal((L, d), dtype=np.float32)

@@ -6,12 +6,14 @@ CPU-baseline leg of bench.py, never by the product path.
 from .vda_ref import (  # noqa: F401
     RMS_EPS,
     batch_rule_update,
+    decayed,
     boundary_states,
     frame_stats,
     frame_update,
     forward_scan,
     reverse_scan,
     gathered_state,
+    gathered_state_frame,
     num_chunks,
     rms_gate,
     text_state,

@@ -15,7 +15,11 @@ Notation (per batch b, head h, interior latent frame t):
   G_t in R^{U x d_v} (gate logits), state S in R^{d_v x d_k}, read as o = S q.
 
 Readings of points the paper leaves open (each is listed in the design notes):
-  * decay alpha == 1 on this path, so S_bar_t = S_{t-1} and no decay bridge;
+  * decay: without `alpha` the gate is 1, so S_bar_t = S_{t-1} and there is no
+    decay bridge; with `alpha` [T, d_k] in [0, 1] (Eq. 2) both scans use
+    S_bar_t = S_{t+-1} Diag(alpha_t) with the frame's own alpha_t, and query
+    frame t reads the bridged states of Eq. A.4; a side without distant frames
+    bridges its initial state over the same frames;
   * chunks tile the interior frame index from 0: chunk c = [cC, cC + C);
     a ragged last chunk is allowed;
   * the window of chunk c is chunks [c - w, c + w], clipped to interior
@@ -112,26 +116,34 @@ def window_bounds(c, T, chunk, window_chunks):
     return lo, hi
 
 
-def forward_scan(S0, A_all, B_all):
-    """Forward states P_t = (P_{t-1} + B_t)(I + A_t)^{-1}, P_{-1} = S0.
-    Returns the list [P_0, ..., P_{T-1}] (Section 2.2; Eq. 5 with alpha = 1)."""
+def decayed(S, alpha_t):
+    """S_bar = S Diag(alpha_t)  (Eq. 2): channel-wise decay of the key columns."""
+    return _f64(S) * _f64(alpha_t)[None, :]
+
+
+def forward_scan(S0, A_all, B_all, alpha=None):
+    """Forward states P_t = (P_{t-1} Diag(alpha_t) + B_t)(I + A_t)^{-1},
+    P_{-1} = S0 (Section 2.2; Eq. 2 and Eq. 5; alpha None means 1).
+    Returns the list [P_0, ..., P_{T-1}]."""
     P = _f64(S0)
     out = []
     for t in range(len(A_all)):
-        P = frame_update(P, A_all[t], B_all[t])
+        S_bar = P if alpha is None else decayed(P, alpha[t])
+        P = frame_update(S_bar, A_all[t], B_all[t])
         out.append(P)
     return out
 
 
-def reverse_scan(S0, A_all, B_all):
-    """Reverse states R_t = (R_{t+1} + B_t)(I + A_t)^{-1}, R_T = S0, the same
-    frame update taken from the last interior frame down.  Returns the list
-    [R_0, ..., R_{T-1}] indexed by frame."""
+def reverse_scan(S0, A_all, B_all, alpha=None):
+    """Reverse states R_t = (R_{t+1} Diag(alpha_t) + B_t)(I + A_t)^{-1},
+    R_T = S0: the same frame update taken from the last interior frame down.
+    Returns the list [R_0, ..., R_{T-1}] indexed by frame."""
     T = len(A_all)
     R = _f64(S0)
     out = [None] * T
     for t in range(T - 1, -1, -1):
-        R = frame_update(R, A_all[t], B_all[t])
+        S_bar = R if alpha is None else decayed(R, alpha[t])
+        R = frame_update(S_bar, A_all[t], B_all[t])
         out[t] = R
     return out
 
@@ -146,6 +158,21 @@ def gathered_state(c, T, chunk, window_chunks, P, R, S0_fwd, S0_rev):
     return left + right
 
 
+def gathered_state_frame(t, T, chunk, window_chunks, P, R, S0_fwd, S0_rev, alpha):
+    """S~_t for query frame t with the decay bridge (Eq. A.4):
+      S~_t = P_{l-1} Diag(prod_{r=l}^{t} alpha_r) + R_{h+1} Diag(prod_{r=t}^{h} alpha_r)
+    with [l, h] the window of t's chunk; a side without distant frames starts
+    from its initial state.  The products are channel-wise."""
+    c = t // chunk
+    lo, hi = window_bounds(c, T, chunk, window_chunks)
+    alpha = _f64(alpha)
+    left = P[lo - 1] if lo > 0 else _f64(S0_fwd)
+    right = R[hi + 1] if hi < T - 1 else _f64(S0_rev)
+    a_left = np.prod(alpha[lo:t + 1], axis=0)
+    a_right = np.prod(alpha[t:hi + 1], axis=0)
+    return left * a_left[None, :] + right * a_right[None, :]
+
+
 def rms_gate(o, g, w, eps=RMS_EPS):
     """Linear-branch epilogue of Eq. (1c): sigmoid(g) * RMSNorm(o), where
     RMSNorm(o) = w * o / sqrt(mean(o^2) + eps) over the last axis (d_v)."""
@@ -157,18 +184,20 @@ def rms_gate(o, g, w, eps=RMS_EPS):
 
 
 def vda_forward_head(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev,
-                     chunk, window_chunks, eps=RMS_EPS, keep=False):
+                     chunk, window_chunks, eps=RMS_EPS, keep=False, alpha=None):
     """Bidirectional VDA for one (batch, head).
 
     q, k: [T, U, d_k]; v, gate: [T, U, d_v]; beta: [T, U]; rms_weight: [d_v];
-    S0_fwd, S0_rev: [d_v, d_k] or None (zero state).
+    S0_fwd, S0_rev: [d_v, d_k] or None (zero state); alpha: [T, d_k] decay
+    gates in [0, 1] or None (no decay).
     Returns y [T, U, d_v] (float64) and, if keep, a dict with A, B, M and the
     per-frame states P, R.
 
-    Steps (Algorithm 1 of the paper, steps 3-7, with alpha = 1):
-      stats (Eq. 3b) -> forward and reverse scans of Eq. 5 -> gather of the
-      out-of-window states (Eq. A.4) -> o = S~ q (Eq. 1a) -> RMSNorm and gate
-      (Eq. 1c).
+    Steps (Algorithm 1 of the paper, steps 3-7):
+      stats (Eq. 3b) -> forward and reverse scans of Eq. 5 (with the decay of
+      Eq. 2 when alpha is given) -> gather of the out-of-window states (Eq. A.4,
+      with its decay bridge when alpha is given) -> o = S~ q (Eq. 1a) ->
+      RMSNorm and gate (Eq. 1c).
     """
     q = _f64(q)
     k = _f64(k)
@@ -185,15 +214,20 @@ def vda_forward_head(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev,
         A_t, B_t = frame_stats(k[t], v[t], beta[t])
         A_all.append(A_t)
         B_all.append(B_t)
-    P = forward_scan(S0_fwd, A_all, B_all)
-    R = reverse_scan(S0_rev, A_all, B_all)
+    P = forward_scan(S0_fwd, A_all, B_all, alpha)
+    R = reverse_scan(S0_rev, A_all, B_all, alpha)
 
     y = np.empty((T, U, d_v))
-    for c in range(num_chunks(T, chunk)):
-        S_tilde = gathered_state(c, T, chunk, window_chunks, P, R, S0_fwd, S0_rev)
-        for t in range(c * chunk, min(T, (c + 1) * chunk)):
-            o = q[t] @ S_tilde.T              # o_u = S~ q_u for every token u
-            y[t] = rms_gate(o, gate[t], rms_weight, eps)
+    if alpha is None:
+        for c in range(num_chunks(T, chunk)):
+            S_tilde = gathered_state(c, T, chunk, window_chunks, P, R, S0_fwd, S0_rev)
+            for t in range(c * chunk, min(T, (c + 1) * chunk)):
+                o = q[t] @ S_tilde.T              # o_u = S~ q_u for every token u
+                y[t] = rms_gate(o, gate[t], rms_weight, eps)
+    else:
+        for t in range(T):
+            S_tilde = gathered_state_frame(t, T, chunk, window_chunks, P, R, S0_fwd, S0_rev, alpha)
+            y[t] = rms_gate(q[t] @ S_tilde.T, gate[t], rms_weight, eps)
     if not keep:
         return y
     M_all = [np.linalg.inv(np.eye(d_k) + A_t) for A_t in A_all]
@@ -216,9 +250,10 @@ def boundary_states(P, R, S0_fwd, S0_rev, T, chunk):
 
 
 def vda_forward(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev,
-                chunk, window_chunks, eps=RMS_EPS, heads=None):
+                chunk, window_chunks, eps=RMS_EPS, heads=None, alpha=None):
     """Whole-tensor wrapper: q, k: [B, H, T, U, d_k]; v, gate: [B, H, T, U, d_v];
-    beta: [B, H, T, U]; S0_*: [B, H, d_v, d_k] or None.
+    beta: [B, H, T, U]; S0_*: [B, H, d_v, d_k] or None; alpha: [B, H, T, d_k]
+    or None.
 
     Streams one (b, h) at a time.  `heads` optionally restricts the work to a
     list of (b, h) pairs; the result then holds only those heads, in order,
@@ -229,8 +264,9 @@ def vda_forward(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev,
     for (b, h) in pairs:
         s0f = None if S0_fwd is None else S0_fwd[b, h]
         s0r = None if S0_rev is None else S0_rev[b, h]
+        a = None if alpha is None else alpha[b, h]
         out.append(vda_forward_head(q[b, h], k[b, h], v[b, h], beta[b, h], gate[b, h],
-                                    rms_weight, s0f, s0r, chunk, window_chunks, eps))
+                                    rms_weight, s0f, s0r, chunk, window_chunks, eps, alpha=a))
     out = np.stack(out)
     if heads is None:
         out = out.reshape((Bn, Hn) + out.shape[1:])
@@ -241,12 +277,15 @@ def vda_forward(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev,
 # A second, independent route: rescan from scratch for every query frame.
 # ---------------------------------------------------------------------------
 def vda_forward_head_naive(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev,
-                           chunk, window_chunks, eps=RMS_EPS):
+                           chunk, window_chunks, eps=RMS_EPS, alpha=None):
     """O(T^2) restatement of Appendix A.3 for small cases: for each query frame
     t, rebuild P_{l_t - 1} by running the forward update over frames
     0..l_t - 1 from S0_fwd, and R_{h_t + 1} by running the reverse update over
     frames T-1..h_t + 1 from S0_rev; statistics are recomputed per token with
-    the summation form of Eq. (3b); no state is reused between queries."""
+    the summation form of Eq. (3b); no state is reused between queries.
+    With alpha, each update first decays its entering state (Eq. 2), and the
+    bridge is taken as the paper describes it, frame by frame: decay without
+    writes over frames l_t..t (forward) and h_t..t (reverse)."""
     q = _f64(q)
     k = _f64(k)
     v = _f64(v)
@@ -272,10 +311,17 @@ def vda_forward_head_naive(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev,
         hi = min(T - 1, (c + window_chunks + 1) * chunk - 1)
         left = S0_fwd.copy()
         for r in range(0, lo):
-            left = frame_update(left, *stats_by_token(r))
+            enter = left if alpha is None else decayed(left, alpha[r])
+            left = frame_update(enter, *stats_by_token(r))
         right = S0_rev.copy()
         for r in range(T - 1, hi, -1):
-            right = frame_update(right, *stats_by_token(r))
+            enter = right if alpha is None else decayed(right, alpha[r])
+            right = frame_update(enter, *stats_by_token(r))
+        if alpha is not None:
+            for r in range(lo, t + 1):
+                left = decayed(left, alpha[r])
+            for r in range(hi, t - 1, -1):
+                right = decayed(right, alpha[r])
         S_t = left + right
         for u in range(U):
             o = S_t @ q[t, u]
