@@ -39,6 +39,7 @@ class VdaArgs(ctypes.Structure):
         ("chunk", c_int), ("window_chunks", c_int),
         ("eps", c_float),
         ("stream", c_void_p),
+        ("alpha", c_void_p),
     ]
 
 

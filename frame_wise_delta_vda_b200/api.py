@@ -44,7 +44,7 @@ def _check_tensor(name, t, dtype=None, shape=None, device=None, allow_none=False
 
 
 def make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks,
-              eps=1e-6, stream=None, check_device=True):
+              eps=1e-6, stream=None, check_device=True, alpha=None):
     """Build the C `vda_args` block from tensors (device or host)."""
     if q.dim() != 5:
         raise ValueError("q must be [B, H, T, U, d_k]")
@@ -64,6 +64,7 @@ def make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, windo
     chk("rms_weight", rms_weight, torch.float32, (d_v,), dev)
     chk("S0_fwd", S0_fwd, torch.float32, (Bn, Hn, d_v, d_k), dev, allow_none=True)
     chk("S0_rev", S0_rev, torch.float32, (Bn, Hn, d_v, d_k), dev, allow_none=True)
+    chk("alpha", alpha, torch.float32, (Bn, Hn, T, d_k), dev, allow_none=True)
     a = VdaArgs()
     a.dtype = dt
     a.q, a.k, a.v, a.beta, a.gate = (t.data_ptr() for t in (q, k, v, beta, gate))
@@ -75,6 +76,7 @@ def make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, windo
     a.chunk, a.window_chunks = int(chunk), int(window_chunks)
     a.eps = float(eps)
     a.stream = _stream(stream).value if check_device else None
+    a.alpha = alpha.data_ptr() if alpha is not None else None
     return a
 
 
@@ -91,17 +93,19 @@ def workspace_for(q, v, chunk):
 
 def vda_forward(q, k, v, beta, gate, rms_weight, S0_fwd=None, S0_rev=None, chunk=5,
                 window_chunks=1, out=None, workspace=None, states_out=None, stats_out=None,
-                eps=1e-6, stream=None):
+                eps=1e-6, stream=None, alpha=None):
     """Bidirectional VDA forward (see include/vda.h).  Returns `out`.
 
-    Without `workspace`, `states_out` or `stats_out` this calls `vda_forward`
-    / `vda_forward_f32` (stream-ordered workspace); otherwise `vda_forward_ex`.
+    Without `workspace`, `states_out`, `stats_out` or `alpha` this calls
+    `vda_forward` / `vda_forward_f32` (stream-ordered workspace); otherwise
+    `vda_forward_ex`.  `alpha` [B, H, T, d_k] float32 adds the decay gate.
     """
     if out is None:
         out = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
-    a = make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks, eps, stream)
+    a = make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks, eps, stream,
+                  alpha=alpha)
     L = lib()
-    if workspace is None and states_out is None and stats_out is None and eps == 1e-6:
+    if workspace is None and states_out is None and stats_out is None and eps == 1e-6 and alpha is None:
         fn = L.vda_forward if a.dtype == VDA_BF16 else L.vda_forward_f32
         rc = fn(a.q, a.k, a.v, a.beta, a.gate, a.rms_weight, a.S0_fwd, a.S0_rev,
                 a.B, a.H, a.T, a.U, a.d_k, a.d_v, a.chunk, a.window_chunks, a.out, a.stream)
@@ -147,15 +151,16 @@ def vda_forward_host_bytes(q, v, chunk):
 
 
 def vda_forward_host(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks,
-                     device_buffer, eps=1e-6):
+                     device_buffer, eps=1e-6, alpha=None):
     """End-to-end forward from host (CPU, ideally pinned) tensors; copies in,
     computes on the current CUDA device and copies `out` back (synchronous)."""
     for name, t in (("q", q), ("k", k), ("v", v), ("beta", beta), ("gate", gate),
-                    ("rms_weight", rms_weight), ("out", out), ("S0_fwd", S0_fwd), ("S0_rev", S0_rev)):
+                    ("rms_weight", rms_weight), ("out", out), ("S0_fwd", S0_fwd), ("S0_rev", S0_rev),
+                    ("alpha", alpha)):
         if t is not None and (t.is_cuda or not t.is_contiguous()):
             raise ValueError(f"{name} must be a contiguous host tensor")
     a = make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks, eps,
-                  check_device=False)
+                  check_device=False, alpha=alpha)
     if not device_buffer.is_cuda:
         raise ValueError("device_buffer must be a CUDA tensor")
     rc = lib().vda_forward_host(ctypes.byref(a), _ptr(device_buffer), device_buffer.numel())
@@ -164,14 +169,15 @@ def vda_forward_host(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk
 
 
 def vda_forward_noalloc(q, k, v, beta, gate, rms_weight, S0_fwd=None, S0_rev=None, chunk=5,
-                        window_chunks=1, out=None, eps=1e-6, stream=None):
+                        window_chunks=1, out=None, eps=1e-6, stream=None, alpha=None):
     """Forward through `vda_forward_noalloc`: the library uses its fixed
     internal scratch array instead of any allocation (sizes must fit in
     NOALLOC_SCRATCH_BYTES of workspace).  `out` must be preallocated by callers
     that cannot allocate; it is created here only as a convenience."""
     if out is None:
         out = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
-    a = make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks, eps, stream)
+    a = make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks, eps, stream,
+                  alpha=alpha)
     check(lib().vda_forward_noalloc(ctypes.byref(a)), "vda_forward_noalloc")
     return out
 

@@ -156,9 +156,11 @@ k_gj_inverse(float* __restrict__ AM) {
 }
 
 // ---------------------------------------------------------------------------
-// Bidirectional scan (Section 2.2; Eq. 5 with alpha = 1), SIMT:
-//   forward  P_t = (P_{t-1} + B_t) M_t  for t = 0..T-1 from S0_fwd
-//   reverse  R_t = (R_{t+1} + B_t) M_t  for t = T-1..0 from S0_rev
+// Bidirectional scan (Section 2.2; Eq. 5, with the decay of Eq. 2 when alpha
+// is given), SIMT:
+//   forward  P_t = (P_{t-1} Diag(alpha_t) + B_t) M_t  for t = 0..T-1 from S0_fwd
+//   reverse  R_t = (R_{t+1} Diag(alpha_t) + B_t) M_t  for t = T-1..0 from S0_rev
+// (alpha NULL: no decay)
 // Right-multiplication acts on each row of S independently, so a chain
 // (b, h, dir) is split over CTAs by blocks of RB rows with no communication.
 // Thread j owns column j of its rows.  Chunk-boundary states are written to
@@ -169,7 +171,7 @@ template <int D, int RB>
 __global__ void __launch_bounds__(D)
 k_scan_simt(const float* __restrict__ M, const float* __restrict__ Bm,
             const float* __restrict__ S0f, const float* __restrict__ S0r,
-            float* __restrict__ states, int BH, int T, int chunk, int NC) {
+            const float* __restrict__ alpha, float* __restrict__ states, int BH, int T, int chunk, int NC) {
   __shared__ float sX[RB][D];
   const int bh = blockIdx.x, dir = blockIdx.y, r0 = blockIdx.z * RB, j = threadIdx.x;
   const size_t DD = (size_t)D * D;
@@ -190,8 +192,14 @@ k_scan_simt(const float* __restrict__ M, const float* __restrict__ Bm,
     const int t = dir == 0 ? step : T - 1 - step;
     const float* Bt = Bm + ((size_t)bh * T + t) * DD;
     const float* Mt = M + ((size_t)bh * T + t) * DD;
+    if (alpha) {   // S_bar = S Diag(alpha_t): thread j holds key column j (Eq. 2)
+      const float a = __ldg(alpha + ((size_t)bh * T + t) * D + j);
 #pragma unroll
-    for (int i = 0; i < RB; ++i) sX[i][j] = s[i] + Bt[(size_t)(r0 + i) * D + j];
+      for (int i = 0; i < RB; ++i) sX[i][j] = fmaf(s[i], a, Bt[(size_t)(r0 + i) * D + j]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < RB; ++i) sX[i][j] = s[i] + Bt[(size_t)(r0 + i) * D + j];
+    }
     __syncthreads();
     float acc[RB];
 #pragma unroll
@@ -220,10 +228,39 @@ k_scan_simt(const float* __restrict__ M, const float* __restrict__ Bm,
 }
 
 // ---------------------------------------------------------------------------
+// Decay bridge of Appendix A.3 (Eq. A.4): for query frame t in chunk c with
+// window [l, h] (chunks c-w .. c+w clipped to the clip),
+//   bridge[b,h,t][0][k] = prod_{r=l..t} alpha_r[k]   (applied to P_{l-1})
+//   bridge[b,h,t][1][k] = prod_{r=t..h} alpha_r[k]   (applied to R_{h+1})
+// One thread per (b, h, t, k).
+// ---------------------------------------------------------------------------
+__global__ void k_decay_bridge(const float* __restrict__ alpha, int BH, int T, int D, int chunk,
+                               int window_chunks, float* __restrict__ bridge) {
+  const size_t n = (size_t)BH * T * D;
+  const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n) return;
+  const int k = (int)(idx % (size_t)D);
+  const size_t ft = idx / (size_t)D;
+  const int t = (int)(ft % (size_t)T);
+  const size_t bh = ft / (size_t)T;
+  const int c = t / chunk;
+  const int lo = max(0, (c - window_chunks) * chunk);
+  const int hi = min(T - 1, (c + window_chunks + 1) * chunk - 1);
+  const float* a = alpha + bh * (size_t)T * D + k;
+  float pl = 1.f, pr = 1.f;
+  for (int r = lo; r <= t; ++r) pl *= __ldg(a + (size_t)r * D);
+  for (int r = t; r <= hi; ++r) pr *= __ldg(a + (size_t)r * D);
+  bridge[(ft * 2) * D + k] = pl;
+  bridge[(ft * 2 + 1) * D + k] = pr;
+}
+
+// ---------------------------------------------------------------------------
 // Readout (Appendix A.3 gather + Eq. 1a + Eq. 1c), SIMT.  One CTA column per
-// (b, h, chunk c); gridDim.y CTAs split the chunk's tokens.  The CTA builds
+// (b, h, chunk c), or per (b, h, frame t) with the decay bridge; gridDim.y
+// CTAs split the unit's tokens.  The CTA builds
 //   S~ = fwd[max(0, c - w)] + rev[min(NC, c + w + 1)]
-// (transposed, in shared memory), then each warp takes groups of tokens:
+// (with the bridge: fwd[..] Diag(bridge[t][0]) + rev[..] Diag(bridge[t][1]))
+// transposed, in shared memory, then each warp takes groups of tokens:
 // G = min(D, 32) lanes per token slot, lane li of a slot computes outputs
 // i = li + G*m; NT tokens per slot share every S~ load.
 //   y = sigmoid(g) * w * o / sqrt(mean(o^2) + eps)
@@ -245,22 +282,34 @@ template <int D, typename TIo>
 __global__ void __launch_bounds__(256)
 k_readout_simt(const TIo* __restrict__ Q, const TIo* __restrict__ Gt,
                const float* __restrict__ w, const float* __restrict__ states,
-               TIo* __restrict__ out, int BH, int T, int U, int chunk, int NC,
-               int window_chunks, float eps) {
+               const float* __restrict__ bridge, TIo* __restrict__ out, int BH, int T, int U, int chunk,
+               int NC, int window_chunks, float eps) {
   using Cfg = ReadoutSimtCfg<D, TIo>;
   extern __shared__ float smem[];
   float* sT = smem;                                       // [D][D], sT[k][i] = S~[i][k]
   float* sQ = smem + (size_t)D * D;                       // [WARPS][TOK_PER_WARP][D]
 
-  const int bh = blockIdx.x / NC, c = blockIdx.x - (blockIdx.x / NC) * NC;
+  // unit = one chunk, or one frame with the decay bridge (its read state
+  // changes from frame to frame)
+  const int NU = bridge ? T : NC;
+  const int bh = blockIdx.x / NU, u = blockIdx.x - (blockIdx.x / NU) * NU;
+  const int c = bridge ? u / chunk : u;
   const size_t DD = (size_t)D * D;
   const int jf = max(0, c - window_chunks);
   const int jr = min(NC, c + window_chunks + 1);
   const float* Sf = states + ((size_t)0 * BH + bh) * (size_t)(NC + 1) * DD + (size_t)jf * DD;
   const float* Sr = states + ((size_t)1 * BH + bh) * (size_t)(NC + 1) * DD + (size_t)jr * DD;
-  for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
-    const int i = e / D, k = e - (e / D) * D;
-    sT[(size_t)k * D + i] = Sf[e] + Sr[e];
+  if (bridge) {
+    const float* al = bridge + (((size_t)bh * T + u) * 2) * D;
+    for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+      const int i = e / D, k = e - (e / D) * D;
+      sT[(size_t)k * D + i] = fmaf(Sf[e], al[k], Sr[e] * al[D + k]);
+    }
+  } else {
+    for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+      const int i = e / D, k = e - (e / D) * D;
+      sT[(size_t)k * D + i] = Sf[e] + Sr[e];
+    }
   }
   __syncthreads();
 
@@ -268,7 +317,7 @@ k_readout_simt(const TIo* __restrict__ Q, const TIo* __restrict__ Gt,
   const int slot = lane / Cfg::G, li = lane - (lane / Cfg::G) * Cfg::G;
   float* myQ = sQ + (size_t)warp * Cfg::TOK_PER_WARP * D;
 
-  const int f0 = c * chunk, f1 = min(T, (c + 1) * chunk);
+  const int f0 = bridge ? u : c * chunk, f1 = bridge ? u + 1 : min(T, (c + 1) * chunk);
   const size_t tok0 = ((size_t)bh * T + f0) * U;          // first token row of the chunk
   const int ntok = (f1 - f0) * U;
   float wv[Cfg::PER];

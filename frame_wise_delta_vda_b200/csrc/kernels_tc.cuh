@@ -655,7 +655,8 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
 
 // ===========================================================================
 // k_scan_tc: one CTA per chain (b, h, direction); S in R^{128 x 128} fp32.
-// Step t: X = S + B_t (fp32), then S <- X M_t computed on the tensor cores as
+// Step t: X = S Diag(alpha_t) + B_t (fp32; Eq. 2, alpha = 1 without decay),
+// then S <- X M_t computed on the tensor cores as
 //   D[j][n] = sum_k M[k][j] X[n][k]  with  M = Mh + Ml,  X = Xh + Xl  (bf16)
 //   D = Mh Xh + Mh Xl + Ml Xh        (the dropped Ml Xl term is ~2^-16 rel.)
 // Right-multiplication acts on each row of S independently, so the 128 rows
@@ -708,7 +709,7 @@ __device__ __forceinline__ uint32_t ximg_offset(int n, int k) {
 
 __global__ void __launch_bounds__(ScanCfg::THREADS, 1)
 k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
-          const float* __restrict__ S0f, const float* __restrict__ S0r,
+          const float* __restrict__ S0f, const float* __restrict__ S0r, const float* __restrict__ alpha,
           float* __restrict__ states, int BH, int T, int chunk, int NC) {
   using C = ScanCfg;
   extern __shared__ uint8_t smem_raw[];
@@ -809,6 +810,8 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
     {
       const int j0 = dir == 0 ? 0 : NC;
       const float* B0 = Bm + ((size_t)bh * T + frame_of(0)) * kDD + (size_t)(64 * h) * kD + j;
+      // decay of the first frame on key column j (Eq. 2); 1 without decay
+      const float a0 = alpha ? __ldg(alpha + ((size_t)bh * T + frame_of(0)) * kD + j) : 1.f;
 #pragma unroll 2
       for (int c = 0; c < 8; ++c) {
         float x[8];
@@ -817,7 +820,7 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
           const int n = 64 * h + 8 * c + e;
           const float s0 = S0 ? __ldg(S0 + (size_t)bh * kDD + (size_t)n * kD + j) : 0.f;
           st[(size_t)j0 * kDD + (size_t)n * kD + j] = s0;
-          x[e] = s0 + __ldg(B0 + (size_t)(8 * c + e) * kD);
+          x[e] = fmaf(s0, a0, __ldg(B0 + (size_t)(8 * c + e) * kD));
         }
         const uint32_t o = xrow + (((uint32_t)c ^ jsw) << 4);
         st_chunk_hilo(o, o + C::XIMG, x);
@@ -834,10 +837,12 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
       } else if (t % chunk == 0) {
         jb = t / chunk;
       }
+      float anext = 1.f;   // decay of the next frame on key column j (Eq. 2)
       if (more) {   // B_{t+1}[64h + n2][j]: 32 lanes read 128 contiguous bytes per row
         const float* Bn = Bm + ((size_t)bh * T + frame_of(i + 1)) * kDD + (size_t)(64 * h) * kD + j;
 #pragma unroll
         for (int n2 = 0; n2 < 64; ++n2) bnext[n2] = __ldg(Bn + (size_t)n2 * kD);
+        if (alpha) anext = __ldg(alpha + ((size_t)bh * T + frame_of(i + 1)) * kD + j);
       }
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(DFULL + h), (uint32_t)i & 1u, abort_flag))) break;
       tc_fence_after();
@@ -855,7 +860,7 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
           for (int q = 0; q < 2; ++q) {
             float x[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(v[8 * q + e]) + bnext[cb * 16 + 8 * q + e];
+            for (int e = 0; e < 8; ++e) x[e] = fmaf(__uint_as_float(v[8 * q + e]), anext, bnext[cb * 16 + 8 * q + e]);
             const uint32_t c8 = (uint32_t)(2 * cb + q);
             const uint32_t o = xrow + ((c8 ^ jsw) << 4);
             st_chunk_hilo(o, o + C::XIMG, x);
@@ -921,28 +926,30 @@ struct ReadoutCfg {
 
 struct ReadoutGeom {
   int BH, T, U, chunk, NC, window;
-  int tpc;         // tiles of a full chunk
-  int tlast;       // tiles of the last chunk
+  int unit;        // frames per unit of equal read state: chunk, or 1 with the decay bridge
+  int NU;          // units per head
+  int tpc;         // tiles of a full unit
+  int tlast;       // tiles of the last unit
   int tph;         // tiles per head
   long long total; // tiles over all heads
 };
 
-// tile index -> (bh, c, first row of the tile relative to the chunk, rows of the chunk)
-__device__ __forceinline__ void tile_coords(const ReadoutGeom& g, long long gt, int& bh, int& c, int& tr, int& rows) {
+// tile index -> (bh, unit u, first row of the tile relative to the unit, rows of the unit)
+__device__ __forceinline__ void tile_coords(const ReadoutGeom& g, long long gt, int& bh, int& u, int& tr, int& rows) {
   bh = (int)(gt / g.tph);
   int rem = (int)(gt - (long long)bh * g.tph);
-  c = rem / g.tpc;
-  if (c > g.NC - 1) c = g.NC - 1;
-  tr = (rem - c * g.tpc) * ReadoutCfg::TILE;
-  const int f0 = c * g.chunk;
-  const int f1 = min(g.T, f0 + g.chunk);
+  u = rem / g.tpc;
+  if (u > g.NU - 1) u = g.NU - 1;
+  tr = (rem - u * g.tpc) * ReadoutCfg::TILE;
+  const int f0 = u * g.unit;
+  const int f1 = min(g.T, f0 + g.unit);
   rows = (f1 - f0) * g.U;
 }
 
 __global__ void __launch_bounds__(ReadoutCfg::THREADS, 1)
 k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
              const __grid_constant__ CUtensorMap tmO,
-             const float* __restrict__ w, const float* __restrict__ states,
+             const float* __restrict__ w, const float* __restrict__ states, const float* __restrict__ bridge,
              __nv_bfloat16* __restrict__ out, ReadoutGeom g, float eps) {
   using C = ReadoutCfg;
   extern __shared__ uint8_t smem_raw[];
@@ -1003,7 +1010,7 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         int bh, c, tr, rows;
         tile_coords(g, gt, bh, c, tr, rows);
         if (tr + C::TILE <= rows) {
-          const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.chunk * g.U + tr);
+          const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.unit * g.U + tr);
           const uint32_t src = base + s * C::TILE_BYTES;
           tma_store_2d(&tmO, src, 0, row0);
           tma_store_2d(&tmO, src + C::TILE_BYTES / 2, 64, row0);
@@ -1015,7 +1022,7 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       for (long long gt = t_begin; gt < t_end; ++gt, ++k) {
         int bh, c, tr, rows;
         tile_coords(g, gt, bh, c, tr, rows);
-        const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.chunk * g.U + tr);
+        const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.unit * g.U + tr);
         const uint32_t s = (uint32_t)(k % ns), ph = (uint32_t)(k / ns) & 1u;
         if (is_q) {
           if (!mbar_wait(BAR(QEMPTY + s), ph ^ 1u, abort_flag)) { ok = false; break; }
@@ -1088,8 +1095,12 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       int bh, c, tr, rows;
       tile_coords(g, gt, bh, c, tr, rows);
       if (bh != prev_bh || c != prev_c) {
-        // build S~ = fwd[max(0, c-w)] + rev[min(NC, c+w+1)]: row i = r, this half's columns
-        const int jf = max(0, c - g.window), jr = min(g.NC, c + g.window + 1);
+        // build S~ = fwd[max(0, c-w)] + rev[min(NC, c+w+1)] (chunk c of this unit),
+        // with the decay bridge fwd Diag(bl) + rev Diag(br) of frame u (Eq. A.4):
+        // row i = r, this half's columns
+        const int cc_ = (c * g.unit) / g.chunk;
+        const int jf = max(0, cc_ - g.window), jr = min(g.NC, cc_ + g.window + 1);
+        const float* bl = bridge ? bridge + (((size_t)bh * g.T + c) * 2) * kD + 64 * ch : nullptr;
         const float* Sf =
             states + (size_t)bh * (size_t)(g.NC + 1) * kDD + (size_t)jf * kDD + (size_t)r * kD + 64 * ch;
         const float* Sr = states + sdir + (size_t)bh * (size_t)(g.NC + 1) * kDD + (size_t)jr * kD * kD +
@@ -1100,8 +1111,18 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
           const float4 f1 = __ldg(reinterpret_cast<const float4*>(Sf + cc * 8 + 4));
           const float4 r0v = __ldg(reinterpret_cast<const float4*>(Sr + cc * 8));
           const float4 r1v = __ldg(reinterpret_cast<const float4*>(Sr + cc * 8 + 4));
-          const float x[8] = {f0.x + r0v.x, f0.y + r0v.y, f0.z + r0v.z, f0.w + r0v.w,
-                              f1.x + r1v.x, f1.y + r1v.y, f1.z + r1v.z, f1.w + r1v.w};
+          float x[8] = {f0.x + r0v.x, f0.y + r0v.y, f0.z + r0v.z, f0.w + r0v.w,
+                        f1.x + r1v.x, f1.y + r1v.y, f1.z + r1v.z, f1.w + r1v.w};
+          if (bl) {
+            const float4 a0 = __ldg(reinterpret_cast<const float4*>(bl + cc * 8));
+            const float4 a1 = __ldg(reinterpret_cast<const float4*>(bl + cc * 8 + 4));
+            const float4 b0 = __ldg(reinterpret_cast<const float4*>(bl + kD + cc * 8));
+            const float4 b1 = __ldg(reinterpret_cast<const float4*>(bl + kD + cc * 8 + 4));
+            x[0] = fmaf(f0.x, a0.x, r0v.x * b0.x); x[1] = fmaf(f0.y, a0.y, r0v.y * b0.y);
+            x[2] = fmaf(f0.z, a0.z, r0v.z * b0.z); x[3] = fmaf(f0.w, a0.w, r0v.w * b0.w);
+            x[4] = fmaf(f1.x, a1.x, r1v.x * b1.x); x[5] = fmaf(f1.y, a1.y, r1v.y * b1.y);
+            x[6] = fmaf(f1.z, a1.z, r1v.z * b1.z); x[7] = fmaf(f1.w, a1.w, r1v.w * b1.w);
+          }
           uint32_t hw[4], lw[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -1162,7 +1183,7 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       // g in place); the chunk's last, partial tile by per-row stores
       const bool tma_out = tr + C::TILE <= rows;
       __nv_bfloat16* orow =
-          out + ((size_t)bh * tokens_per_head + (size_t)c * g.chunk * g.U + tr + r) * kD + 64 * ch;
+          out + ((size_t)bh * tokens_per_head + (size_t)c * g.unit * g.U + tr + r) * kD + 64 * ch;
 #pragma unroll
       for (int cb = 0; cb < 2; ++cb) {   // 4 chunks of 8 columns at a time, loads first
         uint4 gv[4];
@@ -1331,25 +1352,31 @@ inline int launch_inverse(const float* A, size_t FH, uint8_t* Mimg, float* M_dbg
   return launch_status("k_inverse_tc");
 }
 
-inline int launch_scan(const uint8_t* Mimg, const float* Bm, const float* S0f, const float* S0r, float* states,
-                       size_t BH, int T, int chunk, int NC, int ndir, cudaStream_t s) {
+inline int launch_scan(const uint8_t* Mimg, const float* Bm, const float* S0f, const float* S0r,
+                       const float* alpha, float* states, size_t BH, int T, int chunk, int NC, int ndir,
+                       cudaStream_t s) {
   if (cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanCfg::SMEM) !=
       cudaSuccess)
     return VDA_ERR_CUDA;
   dim3 grid((unsigned)BH, (unsigned)ndir);
-  k_scan_tc<<<grid, ScanCfg::THREADS, ScanCfg::SMEM, s>>>(Mimg, Bm, S0f, S0r, states, (int)BH, T, chunk, NC);
+  k_scan_tc<<<grid, ScanCfg::THREADS, ScanCfg::SMEM, s>>>(Mimg, Bm, S0f, S0r, alpha, states, (int)BH, T, chunk,
+                                                          NC);
   return launch_status("k_scan_tc");
 }
 
-inline int launch_readout(const void* Q, const void* G, const float* w, const float* states, void* out,
-                          size_t BH, int T, int U, int chunk, int NC, int window, float eps, cudaStream_t s) {
+inline int launch_readout(const void* Q, const void* G, const float* w, const float* states, const float* bridge,
+                          void* out, size_t BH, int T, int U, int chunk, int NC, int window, float eps,
+                          cudaStream_t s) {
   ReadoutGeom g{};
   g.BH = (int)BH; g.T = T; g.U = U; g.chunk = chunk; g.NC = NC; g.window = window;
-  const long long rows_full = (long long)std::min(T, chunk) * U;
-  const long long rows_last = (long long)(T - (NC - 1) * chunk) * U;
+  // with the decay bridge the read state changes every frame: one unit per frame
+  g.unit = bridge ? 1 : chunk;
+  g.NU = (T + g.unit - 1) / g.unit;
+  const long long rows_full = (long long)std::min(T, g.unit) * U;
+  const long long rows_last = (long long)(T - (g.NU - 1) * g.unit) * U;
   g.tpc = (int)((rows_full + ReadoutCfg::TILE - 1) / ReadoutCfg::TILE);
   g.tlast = (int)((rows_last + ReadoutCfg::TILE - 1) / ReadoutCfg::TILE);
-  g.tph = (NC - 1) * g.tpc + g.tlast;
+  g.tph = (g.NU - 1) * g.tpc + g.tlast;
   g.total = (long long)BH * g.tph;
   const uint64_t rows = (uint64_t)BH * T * U;
   CUtensorMap tmQ, tmG, tmO;
@@ -1361,7 +1388,7 @@ inline int launch_readout(const void* Q, const void* G, const float* w, const fl
     return VDA_ERR_CUDA;
   const int grid = (int)std::min<long long>(g.total, (long long)num_sms());
   k_readout_tc<<<grid, ReadoutCfg::THREADS, ReadoutCfg::SMEM, s>>>(
-      tmQ, tmG, tmO, w, states, static_cast<__nv_bfloat16*>(out), g, eps);
+      tmQ, tmG, tmO, w, states, bridge, static_cast<__nv_bfloat16*>(out), g, eps);
   return launch_status("k_readout_tc");
 }
 
@@ -1382,7 +1409,8 @@ inline int tc_launches_per_forward() { return 4; }
 
 template <typename MarkFn>
 int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_args& a, char* ws_AM,
-              char* ws_B, char* ws_states, char* ws_img, cudaStream_t s, float* stats_out, MarkFn mark) {
+              char* ws_B, char* ws_states, char* ws_img, char* ws_bridge, cudaStream_t s, float* stats_out,
+              MarkFn mark) {
   const size_t FH = BH * (size_t)T;
   const size_t fdd = FH * tc::kDD;
   float* A = reinterpret_cast<float*>(ws_AM);
@@ -1401,12 +1429,20 @@ int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_
   if ((rc = tc::launch_inverse(A, FH, img, stats_out ? stats_out + 2 * fdd : nullptr, s)) != VDA_OK) return rc;
   if ((rc = debug_check("inverse", s)) != VDA_OK) return rc;
   mark(2);
-  if ((rc = tc::launch_scan(img, Bt, a.S0_fwd, a.S0_rev, st, BH, T, chunk, NC, 2, s)) != VDA_OK) return rc;
+  if ((rc = tc::launch_scan(img, Bt, a.S0_fwd, a.S0_rev, a.alpha, st, BH, T, chunk, NC, 2, s)) != VDA_OK)
+    return rc;
   if ((rc = debug_check("scan", s)) != VDA_OK) return rc;
+  float* bridge = nullptr;
+  if (a.alpha) {   // products of the decay bridge (Eq. A.4), one per (b, h, frame, key channel)
+    bridge = reinterpret_cast<float*>(ws_bridge);
+    const size_t n = FH * (size_t)tc::kD;
+    k_decay_bridge<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.alpha, (int)BH, T, tc::kD, chunk, window, bridge);
+    if ((rc = launch_status("k_decay_bridge")) != VDA_OK) return rc;
+  }
   mark(3);
   const float eps = a.eps > 0.f ? a.eps : 1e-6f;
-  if ((rc = tc::launch_readout(a.q, a.gate, a.rms_weight, st, a.out, BH, T, U, chunk, NC, window, eps, s)) !=
-      VDA_OK)
+  if ((rc = tc::launch_readout(a.q, a.gate, a.rms_weight, st, bridge, a.out, BH, T, U, chunk, NC, window, eps,
+                               s)) != VDA_OK)
     return rc;
   if ((rc = debug_check("readout", s)) != VDA_OK) return rc;
   mark(4);
@@ -1423,7 +1459,8 @@ inline int tc_text_state(size_t BH, int L, const void* k, const void* v, const f
   int rc;
   if ((rc = tc::launch_stats(k, v, beta, L, BH, A, Bt, s)) != VDA_OK) return rc;
   if ((rc = tc::launch_inverse(A, BH, img, nullptr, s)) != VDA_OK) return rc;
-  return tc::launch_scan(img, Bt, nullptr, nullptr, reinterpret_cast<float*>(ws_states), BH, 1, 1, 1, 1, s);
+  return tc::launch_scan(img, Bt, nullptr, nullptr, nullptr, reinterpret_cast<float*>(ws_states), BH, 1, 1, 1, 1,
+                         s);
 }
 
 }  // namespace vda

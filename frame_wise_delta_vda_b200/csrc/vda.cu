@@ -35,7 +35,7 @@ struct Plan {
   int B, H, T, U, d, chunk, window, NC, dtype;
   size_t BH, FH;
   bool tc;               // tensor-core (tcgen05) kernels
-  size_t off_AM, off_B, off_states, total;
+  size_t off_AM, off_B, off_states, off_bridge, total;
 };
 
 int check_sizes(int B, int H, int T, int U, int d_k, int d_v, int chunk, int window, int dtype) {
@@ -64,6 +64,7 @@ Plan make_plan(int B, int H, int T, int U, int d, int chunk, int window, int dty
   p.off_AM = off;     off = align_up(off + p.FH * dd);
   p.off_B = off;      off = align_up(off + p.FH * dd);
   p.off_states = off; off = align_up(off + 2 * p.BH * (size_t)(p.NC + 1) * dd);
+  p.off_bridge = off; off = align_up(off + 2 * p.FH * (size_t)d * sizeof(float));   // decay bridge products
   p.total = off + vda::tc_extra_workspace_bytes(p.tc, p.FH, d);
   return p;
 }
@@ -96,6 +97,7 @@ int launch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, int 
   float* Bm = reinterpret_cast<float*>(ws + p.off_B);
   float* st = reinterpret_cast<float*>(ws + p.off_states);
   const size_t fdd = p.FH * (size_t)D * D;
+  float* bridge = a.alpha ? reinterpret_cast<float*>(ws + p.off_bridge) : nullptr;
 
   timing_mark(tslot, 0, s);
   vda::k_stats_simt<D, TIo><<<(unsigned)p.FH, 256, 0, s>>>(
@@ -116,18 +118,26 @@ int launch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, int 
   timing_mark(tslot, 2, s);
   constexpr int RB = 16;
   dim3 gs((unsigned)p.BH, 2, D / RB);
-  vda::k_scan_simt<D, RB><<<gs, D, 0, s>>>(AM, Bm, a.S0_fwd, a.S0_rev, st, (int)p.BH, p.T,
+  vda::k_scan_simt<D, RB><<<gs, D, 0, s>>>(AM, Bm, a.S0_fwd, a.S0_rev, a.alpha, st, (int)p.BH, p.T,
                                            p.chunk, p.NC);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
   timing_mark(tslot, 3, s);
+  if (bridge) {
+    const size_t n = p.FH * (size_t)D;
+    vda::k_decay_bridge<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.alpha, (int)p.BH, p.T, D, p.chunk, p.window,
+                                                                    bridge);
+    if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  }
 
   using Cfg = ReadoutSimtCfg<D, TIo>;
   const size_t smem = Cfg::smem_bytes();
   if (cudaFuncSetAttribute(vda::k_readout_simt<D, TIo>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return VDA_ERR_CUDA;
-  const size_t pairs = p.BH * p.NC;
-  const long long tok_chunk = (long long)std::min(p.T, p.chunk) * p.U;
+  // tokens are taken per chunk, or per frame when the decay bridge makes the
+  // read state differ from frame to frame
+  const size_t pairs = p.BH * (size_t)(bridge ? p.T : p.NC);
+  const long long tok_chunk = (long long)(bridge ? 1 : std::min(p.T, p.chunk)) * p.U;
   const long long per_cta = (long long)Cfg::WARPS * Cfg::TOK_PER_WARP * 4;
   int splits = (int)std::min<long long>((tok_chunk + per_cta - 1) / per_cta,
                                         std::max<long long>(1, 1184 / (long long)pairs));
@@ -135,7 +145,7 @@ int launch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, int 
   dim3 gr((unsigned)pairs, (unsigned)splits);
   const float eps = a.eps > 0.f ? a.eps : 1e-6f;
   vda::k_readout_simt<D, TIo><<<gr, 256, smem, s>>>(
-      static_cast<const TIo*>(a.q), static_cast<const TIo*>(a.gate), a.rms_weight, st,
+      static_cast<const TIo*>(a.q), static_cast<const TIo*>(a.gate), a.rms_weight, st, bridge,
       static_cast<TIo*>(a.out), (int)p.BH, p.T, p.U, p.chunk, p.NC, p.window, eps);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
   timing_mark(tslot, 4, s);
@@ -160,7 +170,8 @@ int validate_args(const vda_args* a) {
   const void* req[] = {a->q, a->k, a->v, a->beta, a->gate, a->rms_weight, a->out};
   for (const void* ptr : req)
     if (!ptr || !aligned16(ptr)) return VDA_ERR_INVALID_ARGUMENT;
-  if ((a->S0_fwd && !aligned16(a->S0_fwd)) || (a->S0_rev && !aligned16(a->S0_rev)))
+  if ((a->S0_fwd && !aligned16(a->S0_fwd)) || (a->S0_rev && !aligned16(a->S0_rev)) ||
+      (a->alpha && !aligned16(a->alpha)))
     return VDA_ERR_INVALID_ARGUMENT;
   return VDA_OK;
 }
@@ -172,7 +183,7 @@ int forward_impl(const vda_args& a, char* ws, const Plan& p, float* states_out, 
   if (p.tc) {
     rc = vda::launch_tc(p.BH, p.T, p.U, p.chunk, p.NC, p.window, a, ws + p.off_AM, ws + p.off_B,
                         ws + p.off_states, ws + p.total - vda::tc_extra_workspace_bytes(true, p.FH, p.d),
-                        s, stats_out,
+                        ws + p.off_bridge, s, stats_out,
                         [&](int stage) { timing_mark(tslot, stage, s); });
   } else if (p.dtype == VDA_BF16) {
     rc = dispatch_simt<__nv_bfloat16>(p, a, ws, s, tslot, stats_out);
@@ -212,7 +223,7 @@ int text_state_simt(const Plan& p, const void* k, const void* v, const float* be
   vda::k_gj_inverse<D><<<(unsigned)p.FH, 256, 0, s>>>(AM);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
   dim3 gs((unsigned)p.BH, 1, D / 16);
-  vda::k_scan_simt<D, 16><<<gs, D, 0, s>>>(AM, Bm, nullptr, nullptr, st, (int)p.BH, 1, 1, p.NC);
+  vda::k_scan_simt<D, 16><<<gs, D, 0, s>>>(AM, Bm, nullptr, nullptr, nullptr, st, (int)p.BH, 1, 1, p.NC);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
   return VDA_OK;
 }
@@ -251,9 +262,9 @@ HostPipe g_pipe[64];
 struct HostLayout {
   int HG, groups;            // heads per group, number of groups
   size_t in_elem;            // bytes per element of q/k/v/gate/out
-  size_t sz_qk, sz_v, sz_beta, sz_s0, sz_w;
+  size_t sz_qk, sz_v, sz_beta, sz_s0, sz_w, sz_alpha;
   size_t slot_off_q, slot_off_k, slot_off_v, slot_off_g, slot_off_beta, slot_off_s0f, slot_off_s0r,
-      slot_off_out, slot_off_ws, slot_bytes;
+      slot_off_alpha, slot_off_out, slot_off_ws, slot_bytes;
   size_t ws_bytes;
   size_t total;
 };
@@ -271,6 +282,7 @@ HostLayout host_layout(int B, int H, int T, int U, int d, int chunk, int dtype) 
   L.sz_beta = tok * sizeof(float);
   L.sz_s0 = (size_t)L.HG * d * d * sizeof(float);
   L.sz_w = (size_t)d * sizeof(float);
+  L.sz_alpha = (size_t)L.HG * T * d * sizeof(float);
   const Plan p = make_plan(1, L.HG, T, U, d, chunk, 0, dtype);
   L.ws_bytes = p.total;
   size_t off = 0;
@@ -281,6 +293,7 @@ HostLayout host_layout(int B, int H, int T, int U, int d, int chunk, int dtype) 
   L.slot_off_beta = off; off = align_up(off + L.sz_beta);
   L.slot_off_s0f = off;  off = align_up(off + L.sz_s0);
   L.slot_off_s0r = off;  off = align_up(off + L.sz_s0);
+  L.slot_off_alpha = off; off = align_up(off + L.sz_alpha);
   L.slot_off_out = off;  off = align_up(off + L.sz_v);
   L.slot_off_ws = off;   off = align_up(off + L.ws_bytes);
   L.slot_bytes = off;
@@ -476,6 +489,9 @@ int vda_forward_host(const vda_args* ha, void* device_buffer, size_t device_byte
       VDA_CK(cudaMemcpyAsync(S + L.slot_off_s0f, ha->S0_fwd + h0 * d * d, s0b, cudaMemcpyHostToDevice, P->h2d));
     if (ha->S0_rev)
       VDA_CK(cudaMemcpyAsync(S + L.slot_off_s0r, ha->S0_rev + h0 * d * d, s0b, cudaMemcpyHostToDevice, P->h2d));
+    if (ha->alpha)
+      VDA_CK(cudaMemcpyAsync(S + L.slot_off_alpha, ha->alpha + h0 * (size_t)ha->T * d,
+                             (size_t)nh * ha->T * d * sizeof(float), cudaMemcpyHostToDevice, P->h2d));
     VDA_CK(cudaEventRecord(P->in_done[sl], P->h2d));
 
     VDA_CK(cudaStreamWaitEvent(P->comp, P->in_done[sl], 0));
@@ -487,6 +503,7 @@ int vda_forward_host(const vda_args* ha, void* device_buffer, size_t device_byte
     a.rms_weight = d_w;
     a.S0_fwd = ha->S0_fwd ? reinterpret_cast<const float*>(S + L.slot_off_s0f) : nullptr;
     a.S0_rev = ha->S0_rev ? reinterpret_cast<const float*>(S + L.slot_off_s0r) : nullptr;
+    a.alpha = ha->alpha ? reinterpret_cast<const float*>(S + L.slot_off_alpha) : nullptr;
     a.out = S + L.slot_off_out;
     a.stream = P->comp;
     const Plan p = make_plan(1, nh, a.T, a.U, d, a.chunk, a.window_chunks, a.dtype);

@@ -3,8 +3,8 @@
  *
  * Paper: "Video DeltaNet: A Video-Native Hybrid Attention for Livestream Video
  * Generation" (arXiv 2609.20744).  The library computes the linear branch of
- * one hybrid attention block (Algorithm 1, steps 3-7, with the decay gate
- * fixed to 1):
+ * one hybrid attention block (Algorithm 1, steps 3-7; shown here with the
+ * decay gate fixed to 1, see "Decay" below for the general form):
  *
  *   for every batch b, head h and interior latent frame t:
  *     A_t = K_t^T Diag(beta_t) K_t,  B_t = V_t^T Diag(beta_t) K_t     (Eq. 3b)
@@ -37,6 +37,16 @@
  *   - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
  *     the legacy default stream) and the call returns without synchronising,
  *     except where stated.
+ *   - Decay (Eq. 2 and Appendix A.3, Eq. A.4): with vda_args.alpha set, both
+ *     scans decay the entering state channel-wise before each frame update,
+ *       P_t = (P_{t-1} Diag(alpha_t) + B_t)(I + A_t)^{-1}   (and R_t alike,
+ *       with the frame's own alpha_t),
+ *     and query frame t reads the bridged states
+ *       S~_t = P_{l-1} Diag(prod_{r=l..t} alpha_r) + R_{h+1} Diag(prod_{r=t..h} alpha_r)
+ *     (a side without distant frames bridges its initial state).  alpha is
+ *     [B, H, T, d_k] float32 with values in [0, 1].  vda_forward and
+ *     vda_forward_f32 have no decay (alpha = 1); vda_forward_ex,
+ *     vda_forward_host and vda_forward_noalloc take it from vda_args.
  *   - Supported sizes: d_k == d_v in {16, 32, 64, 128}; chunk >= 1;
  *     window_chunks >= 0; B, H, T, U >= 1.  d = 128 with bf16 I/O runs on the
  *     tcgen05 tensor-core kernels; the other sizes run on SIMT kernels.
@@ -90,6 +100,7 @@ typedef struct vda_args {
   int window_chunks;          /* window radius in chunks (the paper: 1) */
   float eps;                  /* RMSNorm epsilon; <= 0 selects 1e-6 */
   void* stream;               /* cudaStream_t */
+  const float* alpha;         /* [B,H,T,d_k] decay gates in [0,1] (Eq. 2), or NULL: no decay */
 } vda_args;
 
 /* Bidirectional VDA forward, bf16 I/O.  Takes its workspace stream-ordered
@@ -187,7 +198,9 @@ VDA_API int vda_device_status(void* stream);
 VDA_API int vda_timing_enable(int max_calls);
 VDA_API int vda_timing_read(float* stage_ms, int n_stages, int* calls);
 
-/* Number of kernel launches one vda_forward_ex call with these sizes makes. */
+/* Number of kernel launches one vda_forward_ex call with these sizes makes
+ * without a decay gate; with vda_args.alpha set the call makes one more (the
+ * bridge products of Eq. A.4). */
 VDA_API int vda_launches_per_forward(int B, int H, int T, int U, int d_k, int d_v, int chunk, int dtype);
 
 /* Human-readable name of a vda_status value. */

@@ -42,11 +42,14 @@ def rel_err(got, want):
 
 
 def oracle_head(x, wl, S0f=None, S0r=None, keep=False, w=None):
-    """Oracle output for one head's generated inputs (dict from head_inputs)."""
+    """Oracle output for one head's generated inputs (dict from head_inputs);
+    the decay gates are used when the inputs carry them."""
+    alpha = x.get("alpha")
     return ref.vda_forward_head(gen.as_f64(x["q"]), gen.as_f64(x["k"]), gen.as_f64(x["v"]),
                                 x["beta"], gen.as_f64(x["gate"]),
                                 gen.rms_weight(wl) if w is None else w,
-                                S0f, S0r, wl.chunk, wl.window_chunks, keep=keep)
+                                S0f, S0r, wl.chunk, wl.window_chunks, keep=keep,
+                                alpha=None if alpha is None else gen.as_f64(alpha))
 
 
 def oracle_text_state(x):
