@@ -147,12 +147,13 @@ def algorithmic(wl):
     FH, U, d, e = wl.frame_heads, wl.U, wl.d, 2 if wl.dtype == "bf16" else 4
     BH, NC = wl.B * wl.H, (wl.T + wl.chunk - 1) // wl.chunk
     dd4 = d * d * 4
+    ab = FH * d * 4 if wl.alpha_mean is not None else 0   # decay gates [B, H, T, d_k] fp32
     return {
         "stats": {"bytes": FH * (2 * U * d * e + 4 * U + 2 * dd4), "flops": FH * 4 * U * d * d},
         "inverse": {"bytes": FH * 2 * dd4, "flops": FH * d ** 3},
-        "scan": {"bytes": 2 * FH * 2 * dd4 + 2 * BH * (NC + 1) * dd4, "flops": 2 * FH * 2 * d ** 3},
+        "scan": {"bytes": 2 * FH * 2 * dd4 + 2 * BH * (NC + 1) * dd4 + 2 * ab, "flops": 2 * FH * 2 * d ** 3},
         "readout": {"bytes": FH * 3 * U * d * e + BH * NC * 2 * dd4 + 4 * d, "flops": FH * 2 * U * d * d},
-        "op": {"bytes": FH * (5 * U * d * e + 4 * U), "flops": FH * (6 * U * d * d + 5 * d ** 3)},
+        "op": {"bytes": FH * (5 * U * d * e + 4 * U) + ab, "flops": FH * (6 * U * d * d + 5 * d ** 3)},
     }
 
 
@@ -193,7 +194,8 @@ def cpu_baseline(wl, budget_s=15.0):
         S0 = ref.text_state(gen.as_f64(x["k_text"]), gen.as_f64(x["v_text"]), x["beta_text"]) \
             if wl.text_tokens else None
         ref.vda_forward_head(gen.as_f64(x["q"]), gen.as_f64(x["k"]), gen.as_f64(x["v"]), x["beta"],
-                             gen.as_f64(x["gate"]), w, S0, S0, wl.chunk, wl.window_chunks)
+                             gen.as_f64(x["gate"]), w, S0, S0, wl.chunk, wl.window_chunks,
+                             alpha=gen.as_f64(x["alpha"]) if "alpha" in x else None)
         t_total += time.perf_counter() - t0
         heads += 1
         h += 1
@@ -209,14 +211,16 @@ def run_reference(args):
     if rank != 0:
         return
     import oracle as ref
-    wl = gen.WORKLOADS[WORKLOAD]
+    wl = gen.WORKLOADS[args.workload]
     x = gen.head_inputs(wl, 0, 0)
     w = gen.rms_weight(wl)
     args_f64 = [gen.as_f64(x["q"]), gen.as_f64(x["k"]), gen.as_f64(x["v"]), x["beta"], gen.as_f64(x["gate"])]
-    S0 = ref.text_state(gen.as_f64(x["k_text"]), gen.as_f64(x["v_text"]), x["beta_text"])
+    S0 = ref.text_state(gen.as_f64(x["k_text"]), gen.as_f64(x["v_text"]), x["beta_text"]) \
+        if wl.text_tokens else None
+    alpha = gen.as_f64(x["alpha"]) if "alpha" in x else None
 
     def step():
-        ref.vda_forward_head(*args_f64, w, S0, S0, wl.chunk, wl.window_chunks)
+        ref.vda_forward_head(*args_f64, w, S0, S0, wl.chunk, wl.window_chunks, alpha=alpha)
 
     for _ in range(args.warmup):
         step()
@@ -235,8 +239,9 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} T={wl.T} U={wl.U} d={wl.d} "
-                                   f"chunk={wl.chunk} window=+-{wl.window_chunks}",
-                       "sample": "one head of 48 per step (oracle, host cores)"},
+                                   f"chunk={wl.chunk} window=+-{wl.window_chunks}"
+                                   + (", decay gate" if alpha is not None else ""),
+                       "sample": f"one head of {wl.B * wl.H} per step (oracle, host cores)"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": "one head of the full workload per step"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -287,9 +292,11 @@ def main():
     ws = api.workspace_for(t["q"], t["v"], wl.chunk)
     stream = torch.cuda.current_stream()
 
+    alpha = t.get("alpha")
+
     def step():
         api.vda_forward(t["q"], t["k"], t["v"], t["beta"], t["gate"], t["rms_weight"], S0, S0,
-                        chunk=wl.chunk, window_chunks=wl.window_chunks, out=out, workspace=ws)
+                        chunk=wl.chunk, window_chunks=wl.window_chunks, out=out, workspace=ws, alpha=alpha)
 
     for _ in range(args.warmup):
         step()
@@ -321,7 +328,9 @@ def main():
     if world > 1:
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
     ms_max = float(ms_t.item())
-    launches = api.vda_launches_per_forward(wl.B, wl.H, wl.T, wl.U, wl.d, wl.d, wl.chunk) * args.steps
+    # a decay gate adds one launch per forward (the bridge products)
+    launches = (api.vda_launches_per_forward(wl.B, wl.H, wl.T, wl.U, wl.d, wl.d, wl.chunk)
+                + (1 if alpha is not None else 0)) * args.steps
 
     # ---- end to end through the host-buffer entry point ------------------------
     e2e_steps = args.e2e_steps if args.e2e_steps is not None else max(3, min(args.steps, 10))
@@ -341,7 +350,7 @@ def run_e2e(api, x, S0, out, wl, dev, e2e_steps, world, dist):
     """End-to-end timing through vda_forward_host with pinned host buffers."""
     import torch
     host = {k: torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).pin_memory()
-            for k, v in x.items() if k in ("q", "k", "v", "gate", "beta", "rms_weight")}
+            for k, v in x.items() if k in ("q", "k", "v", "gate", "beta", "rms_weight", "alpha")}
     for k in ("q", "k", "v", "gate"):
         host[k] = host[k].view(torch.bfloat16)
     S0_host = S0.cpu().pin_memory() if S0 is not None else None
@@ -350,7 +359,7 @@ def run_e2e(api, x, S0, out, wl, dev, e2e_steps, world, dist):
 
     def e2e_step():
         api.vda_forward_host(host["q"], host["k"], host["v"], host["beta"], host["gate"], host["rms_weight"],
-                             S0_host, S0_host, out_host, wl.chunk, wl.window_chunks, hbuf)
+                             S0_host, S0_host, out_host, wl.chunk, wl.window_chunks, hbuf, alpha=host.get("alpha"))
 
     e2e_step()
     if not torch.equal(out_host.view(torch.int16), out.cpu().view(torch.int16)):
@@ -406,7 +415,9 @@ def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} T={wl.T} U={wl.U} d={wl.d} chunk={wl.chunk} "
                                f"window=+-{wl.window_chunks}"
-                               + (f", text S0 from {wl.text_tokens} prompt tokens" if wl.text_tokens else ", S0 = 0"),
+                               + (f", text S0 from {wl.text_tokens} prompt tokens" if wl.text_tokens else ", S0 = 0")
+                               + (f", decay gate alpha = sigmoid(N({wl.alpha_mean}, 1))" if wl.alpha_mean is not None
+                                  else ""),
                    "per_rank_problem": "independent problem of the same size per GPU",
                    "l2": "inputs larger than L2 (about 3 GB read per step), no flush",
                    "parallelism": f"replicas{world}"},

@@ -927,6 +927,7 @@ struct ReadoutCfg {
 struct ReadoutGeom {
   int BH, T, U, chunk, NC, window;
   int unit;        // frames per unit of equal read state: chunk, or 1 with the decay bridge
+  int frame_out;   // output map is [frames][U][128]: every tile of a one-frame unit leaves by TMA
   int NU;          // units per head
   int tpc;         // tiles of a full unit
   int tlast;       // tiles of the last unit
@@ -1009,9 +1010,14 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       auto store_out = [&](long long gt, uint32_t s) {
         int bh, c, tr, rows;
         tile_coords(g, gt, bh, c, tr, rows);
-        if (tr + C::TILE <= rows) {
+        const uint32_t src = base + s * C::TILE_BYTES;
+        if (g.frame_out) {   // rows past the frame's U are outside the map: not written
+          const int fh = bh * g.T + c;
+          tma_store_3d(&tmO, src, 0, tr, fh);
+          tma_store_3d(&tmO, src + C::TILE_BYTES / 2, 64, tr, fh);
+          bulk_commit_group();
+        } else if (tr + C::TILE <= rows) {
           const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.unit * g.U + tr);
-          const uint32_t src = base + s * C::TILE_BYTES;
           tma_store_2d(&tmO, src, 0, row0);
           tma_store_2d(&tmO, src + C::TILE_BYTES / 2, 64, row0);
           bulk_commit_group();
@@ -1181,7 +1187,7 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       const bool valid = tr + r < rows;
       // a tile inside its chunk leaves by TMA from the gate stage (y replaces
       // g in place); the chunk's last, partial tile by per-row stores
-      const bool tma_out = tr + C::TILE <= rows;
+      const bool tma_out = g.frame_out || tr + C::TILE <= rows;
       __nv_bfloat16* orow =
           out + ((size_t)bh * tokens_per_head + (size_t)c * g.unit * g.U + tr + r) * kD + 64 * ch;
 #pragma unroll
@@ -1369,8 +1375,10 @@ inline int launch_readout(const void* Q, const void* G, const float* w, const fl
                           cudaStream_t s) {
   ReadoutGeom g{};
   g.BH = (int)BH; g.T = T; g.U = U; g.chunk = chunk; g.NC = NC; g.window = window;
-  // with the decay bridge the read state changes every frame: one unit per frame
+  // with the decay bridge the read state changes every frame: one unit per frame,
+  // and the output map is 3-D by frame so that TMA clips each frame's last tile
   g.unit = bridge ? 1 : chunk;
+  g.frame_out = bridge ? 1 : 0;
   g.NU = (T + g.unit - 1) / g.unit;
   const long long rows_full = (long long)std::min(T, g.unit) * U;
   const long long rows_last = (long long)(T - (g.NU - 1) * g.unit) * U;
@@ -1380,8 +1388,9 @@ inline int launch_readout(const void* Q, const void* G, const float* w, const fl
   g.total = (long long)BH * g.tph;
   const uint64_t rows = (uint64_t)BH * T * U;
   CUtensorMap tmQ, tmG, tmO;
-  if (!encode_bf16_2d(&tmQ, Q, rows, ReadoutCfg::TILE) || !encode_bf16_2d(&tmG, G, rows, ReadoutCfg::TILE) ||
-      !encode_bf16_2d(&tmO, out, rows, ReadoutCfg::TILE))
+  const bool okO = g.frame_out ? encode_bf16_3d(&tmO, out, (uint64_t)U, (uint64_t)BH * T, ReadoutCfg::TILE)
+                               : encode_bf16_2d(&tmO, out, rows, ReadoutCfg::TILE);
+  if (!encode_bf16_2d(&tmQ, Q, rows, ReadoutCfg::TILE) || !encode_bf16_2d(&tmG, G, rows, ReadoutCfg::TILE) || !okO)
     return VDA_ERR_CUDA;
   if (cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ReadoutCfg::SMEM) !=
       cudaSuccess)
