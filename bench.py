@@ -35,6 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from frame_wise_delta_vda_b200 import inputs as gen  # noqa: E402
+from frame_wise_delta_vda_b200 import ranks  # noqa: E402
 
 WORKLOAD = "full"
 METRIC = "VDA fwd+rev frame-tokens/s at H=48,U=1008,d=128; % of HBM/tensor roofline"
@@ -275,7 +276,7 @@ def main():
 
     base = gen.WORKLOADS[args.workload]
     # every rank runs its own problem of the same size (weak scaling)
-    wl = gen.Workload(**{**base.__dict__, "seed": base.seed + 1000 * rank})
+    wl = gen.Workload(**{**base.__dict__, "seed": ranks.rank_seed(base.seed, rank)})
 
     x = gen.make_inputs(wl)
     if "k_text" not in x:
@@ -324,10 +325,7 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
 
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = ranks.max_over_ranks(ms, dist if world > 1 else None, dev)
     # a decay gate adds one launch per forward (the bridge products)
     launches = (api.vda_launches_per_forward(wl.B, wl.H, wl.T, wl.U, wl.d, wl.d, wl.chunk)
                 + (1 if alpha is not None else 0)) * args.steps
@@ -372,10 +370,7 @@ def run_e2e(api, x, S0, out, wl, dev, e2e_steps, world, dist):
         e2e_step()
     torch.cuda.synchronize()
     e2e_s = (time.perf_counter() - t0) / e2e_steps
-    e2e_t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_s = float(e2e_t.item())
+    e2e_s = ranks.max_over_ranks(e2e_s, dist if world > 1 else None, dev)
     h2d = sum(int(host[k].numel() * host[k].element_size()) for k in host)
     if S0_host is not None:
         h2d += 2 * S0_host.numel() * 4
