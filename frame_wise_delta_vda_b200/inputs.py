@@ -185,3 +185,69 @@ def as_f64(x):
     if x.dtype == np.uint16:
         return bf16_bits_to_f32(x).astype(np.float64)
     return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Feature preparation (VDA-Prep) inputs: the QKV projections of the interior
+# video tokens, before the linear branch's feature map, and its filters.
+# ---------------------------------------------------------------------------
+_PQ, _PK, _PV, _PWKS, _PWKT, _PWVS, _PWVT = range(20, 27)
+
+
+@dataclass(frozen=True)
+class PrepWorkload:
+    name: str
+    B: int
+    H: int
+    T: int           # interior latent frames
+    Hl: int          # latent grid rows
+    Wl: int          # latent grid columns (tokens per frame U = Hl * Wl)
+    d: int
+    seed: int
+
+    @property
+    def U(self):
+        return self.Hl * self.Wl
+
+    @property
+    def tokens(self):
+        return self.B * self.T * self.U
+
+
+PREP_WORKLOADS = {
+    "prep_small": PrepWorkload("prep_small", 1, 4, 6, 6, 8, 64, 21),
+    "prep_odd": PrepWorkload("prep_odd", 2, 3, 5, 3, 7, 128, 22),
+    # the full-size shapes: 60 interior frames of a 24 x 42 latent grid
+    "prep_full": PrepWorkload("prep_full", 1, 48, 60, 24, 42, 128, 23),
+}
+
+
+def prep_head_inputs(pw: PrepWorkload, b: int, h: int):
+    """Raw q, k, v of one (batch, head) as [T, U, d] bf16 bits (N(0,1) draws),
+    and the head's filters: wk_s, wv_s [d, 5, 5] ~ N(0, 0.2^2) and wk_t, wv_t
+    [d, 5] ~ N(0, 0.45^2) (float32)."""
+    T, U, d = pw.T, pw.U, pw.d
+    out = {}
+    for key, sid in (("q", _PQ), ("k", _PK), ("v", _PV)):
+        out[key] = f32_to_bf16_bits(_rng(pw.seed, sid, b, h).standard_normal((T, U, d), dtype=np.float32))
+    for key, sid in (("wk_s", _PWKS), ("wv_s", _PWVS)):
+        out[key] = (np.float32(0.2) * _rng(pw.seed, sid, 0, h).standard_normal((d, 5, 5), dtype=np.float32))
+    for key, sid in (("wk_t", _PWKT), ("wv_t", _PWVT)):
+        out[key] = (np.float32(0.45) * _rng(pw.seed, sid, 0, h).standard_normal((d, 5), dtype=np.float32))
+    return out
+
+
+def make_prep_inputs(pw: PrepWorkload):
+    """All prep inputs: q, k, v [B, T, U, H, d] (bf16 bits, heads inner, as a
+    projection lays them out) and the filters wk_s, wv_s [H, d, 5, 5],
+    wk_t, wv_t [H, d, 5] (float32; filters are per head, shared by batches)."""
+    per = {(b, h): prep_head_inputs(pw, b, h) for b in range(pw.B) for h in range(pw.H)}
+    out = {}
+    for key in ("q", "k", "v"):
+        arr = np.empty((pw.B, pw.T, pw.U, pw.H, pw.d), dtype=np.uint16)
+        for (b, h), x in per.items():
+            arr[b, :, :, h, :] = x[key]
+        out[key] = arr
+    for key in ("wk_s", "wk_t", "wv_s", "wv_t"):
+        out[key] = np.ascontiguousarray(np.stack([per[(0, h)][key] for h in range(pw.H)]))
+    return out

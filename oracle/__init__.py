@@ -22,3 +22,13 @@ from .vda_ref import (  # noqa: F401
     vda_forward_head_naive,
     window_bounds,
 )
+from .prep_ref import (  # noqa: F401
+    L2_EPS,
+    conv_spatial,
+    conv_temporal,
+    l2_normalize,
+    prep,
+    prep_head,
+    short_conv,
+    silu,
+)
