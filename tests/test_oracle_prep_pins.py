@@ -137,3 +137,23 @@ def test_grid_transpose_symmetry():
     Xt = X.transpose(0, 2, 1, 3).copy()
     b = ref.short_conv(Xt.reshape(T, Wl * Hl, d), ws.transpose(0, 2, 1), wt, Wl, Hl).reshape(T, Wl, Hl, d)
     np.testing.assert_allclose(b.transpose(0, 2, 1, 3), a, atol=1e-12)
+
+
+def test_scaled_centre_taps_apply_silu_after_the_filter():
+    """Centre taps a (spatial) and b (temporal) scale the input by a*b, so the
+    features are L2(SiLU(a b k)) and SiLU(a b v): the nonlinearity follows the
+    convolution (SiLU(3x) differs from 3 SiLU(x))."""
+    pw = gen.PrepWorkload("scaled", 1, 2, 3, 2, 3, 4, 8)
+    x = gen.make_prep_inputs(pw)
+    s = np.zeros((pw.H, pw.d, 5, 5))
+    s[:, :, 2, 2] = 1.5
+    t = np.zeros((pw.H, pw.d, 5))
+    t[:, :, 2] = 2.0
+    q, k, v = (gen.as_f64(x[n]) for n in ("q", "k", "v"))
+    _, ko, vo = ref.prep(q, k, v, s, t, s, t, pw.Hl, pw.Wl)
+    for h in range(pw.H):
+        k3 = 3.0 * k[0, :, :, h]
+        sk = k3 / (1 + np.exp(-k3))
+        np.testing.assert_allclose(ko[0, h], sk / np.sqrt((sk ** 2).sum(-1, keepdims=True) + ref.L2_EPS), atol=1e-13)
+        v3 = 3.0 * v[0, :, :, h]
+        np.testing.assert_allclose(vo[0, h], v3 / (1 + np.exp(-v3)), atol=1e-13)
