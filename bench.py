@@ -56,6 +56,8 @@ def parse():
                     help="workload to run (the benchmark line is defined on 'full'; other "
                          "workloads serve profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prep", action="store_true",
+                    help="time the feature preparation (vda_prep) on the full-size shapes instead of the forward")
     return ap.parse_args()
 
 
@@ -250,10 +252,74 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------
+def run_prep(args):
+    """One JSON line for the feature preparation step (vda_prep) at the
+    full-size shapes: device time with CUDA events, HBM roofline of its
+    algorithmic bytes (q, k, v in and out, bf16), and the float64 oracle on
+    one head of the host as the CPU baseline."""
+    import torch
+    from frame_wise_delta_vda_b200 import api
+    from frame_wise_delta_vda_b200._lib import lib
+    lib()
+    pw = gen.PREP_WORKLOADS["prep_full"]
+    x = gen.make_prep_inputs(pw)
+
+    def dev_t(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+        return torch.from_numpy(a).cuda()
+
+    t = {k: dev_t(v) for k, v in x.items()}
+    outs = api.vda_prep(t["q"], t["k"], t["v"], t["wk_s"], t["wk_t"], t["wv_s"], t["wv_t"], pw.Hl, pw.Wl)
+
+    def step():
+        api.vda_prep(t["q"], t["k"], t["v"], t["wk_s"], t["wk_t"], t["wv_s"], t["wv_t"], pw.Hl, pw.Wl, *outs)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = min(args.steps, 50)
+    sampler = ClockSampler(0)
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / steps
+    peaks, peak_src = load_peaks()
+    byts = 6 * pw.B * pw.T * pw.U * pw.H * pw.d * 2 + 2 * pw.H * pw.d * 30 * 4
+    ach = byts / (ms * 1e-3) / 1e9
+    line = {"metric": "VDA-Prep frame-tokens/s", "value": pw.tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": 1,
+            "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{pw.name}: B={pw.B} H={pw.H} T={pw.T} grid={pw.Hl}x{pw.Wl} d={pw.d}",
+                       "l2": "inputs larger than L2 (2.2 GB read per step), no flush"},
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"], "traffic": None, "kernel": "k_prep_kv + k_prep_q",
+                         "algorithmic_per_launch": byts, "peak_source": f"hbm_gbs ({peak_src})"},
+            "clocks": clocks, "gpu_launches": 2 * steps}
+    if not args.no_cpu_baseline:
+        import oracle as ref
+        h0 = time.perf_counter()
+        ref.prep(gen.as_f64(x["q"]), gen.as_f64(x["k"]), gen.as_f64(x["v"]), x["wk_s"], x["wk_t"], x["wv_s"],
+                 x["wv_t"], pw.Hl, pw.Wl, heads=[(0, 0)])
+        dt = time.perf_counter() - h0
+        line["cpu_baseline"] = {"value": pw.tokens / pw.H / dt, "unit": UNIT, "kind": "oracle",
+                                "cores": os.cpu_count(),
+                                "sample": f"one head of {pw.H}, fp64 NumPy, {dt:.1f} s; value scaled to all heads"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.prep:
+        run_prep(args)
         return
 
     import torch

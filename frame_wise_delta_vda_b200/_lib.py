@@ -43,6 +43,18 @@ class VdaArgs(ctypes.Structure):
     ]
 
 
+class VdaPrepArgs(ctypes.Structure):
+    """Mirror of `vda_prep_args` in include/vda.h."""
+    _fields_ = [
+        ("q_in", c_void_p), ("k_in", c_void_p), ("v_in", c_void_p),
+        ("wk_s", c_void_p), ("wk_t", c_void_p), ("wv_s", c_void_p), ("wv_t", c_void_p),
+        ("q_out", c_void_p), ("k_out", c_void_p), ("v_out", c_void_p),
+        ("B", c_int), ("H", c_int), ("T", c_int), ("Hl", c_int), ("Wl", c_int), ("d", c_int),
+        ("eps", c_float),
+        ("stream", c_void_p),
+    ]
+
+
 _SIGNATURES = {
     "vda_forward": (c_int, [c_void_p] * 8 + [c_int] * 8 + [c_void_p, c_void_p]),
     "vda_forward_f32": (c_int, [c_void_p] * 8 + [c_int] * 8 + [c_void_p, c_void_p]),
@@ -59,6 +71,7 @@ _SIGNATURES = {
     "vda_timing_read": (c_int, [c_float_p, c_int, c_int_p]),
     "vda_launches_per_forward": (c_int, [c_int] * 8),
     "vda_status_string": (ctypes.c_char_p, [c_int]),
+    "vda_prep": (c_int, [ctypes.POINTER(VdaPrepArgs)]),
 }
 
 _lib = None

@@ -11,7 +11,7 @@ import ctypes
 
 import torch
 
-from ._lib import VDA_BF16, VDA_F32, VdaArgs, VdaError, check, lib  # noqa: F401
+from ._lib import VDA_BF16, VDA_F32, VdaArgs, VdaError, VdaPrepArgs, check, lib  # noqa: F401
 
 _DTYPES = {torch.bfloat16: VDA_BF16, torch.float32: VDA_F32}
 
@@ -120,6 +120,42 @@ def vda_forward(q, k, v, beta, gate, rms_weight, S0_fwd=None, S0_rev=None, chunk
                           _ptr(states_out), _ptr(stats_out))
     check(rc, "vda_forward_ex")
     return out
+
+
+def vda_prep(q_in, k_in, v_in, wk_s, wk_t, wv_s, wv_t, Hl, Wl, q_out=None, k_out=None, v_out=None,
+             eps=1e-6, stream=None):
+    """Feature preparation of the linear branch (see include/vda.h):
+    q_in, k_in, v_in [B, T, U, H, d] bf16 (U = Hl * Wl) -> q', k', v'
+    [B, H, T, U, d] bf16 with q' = L2(q), k' = L2(SiLU(conv(k))),
+    v' = SiLU(conv(v)); filters wk_s, wv_s [H, d, 5, 5], wk_t, wv_t [H, d, 5]
+    float32.  Returns (q_out, k_out, v_out)."""
+    if q_in.dim() != 5:
+        raise ValueError("q_in must be [B, T, U, H, d]")
+    Bn, T, U, Hn, d = q_in.shape
+    if U != Hl * Wl:
+        raise ValueError(f"U = {U} is not Hl * Wl = {Hl} * {Wl}")
+    dev = q_in.device
+    for name, t in (("q_in", q_in), ("k_in", k_in), ("v_in", v_in)):
+        _check_tensor(name, t, torch.bfloat16, (Bn, T, U, Hn, d), dev)
+    for name, t in (("wk_s", wk_s), ("wv_s", wv_s)):
+        _check_tensor(name, t, torch.float32, (Hn, d, 5, 5), dev)
+    for name, t in (("wk_t", wk_t), ("wv_t", wv_t)):
+        _check_tensor(name, t, torch.float32, (Hn, d, 5), dev)
+    outs = []
+    for name, t in (("q_out", q_out), ("k_out", k_out), ("v_out", v_out)):
+        if t is None:
+            t = torch.empty((Bn, Hn, T, U, d), dtype=torch.bfloat16, device=dev)
+        _check_tensor(name, t, torch.bfloat16, (Bn, Hn, T, U, d), dev)
+        outs.append(t)
+    a = VdaPrepArgs()
+    a.q_in, a.k_in, a.v_in = q_in.data_ptr(), k_in.data_ptr(), v_in.data_ptr()
+    a.wk_s, a.wk_t, a.wv_s, a.wv_t = wk_s.data_ptr(), wk_t.data_ptr(), wv_s.data_ptr(), wv_t.data_ptr()
+    a.q_out, a.k_out, a.v_out = (t.data_ptr() for t in outs)
+    a.B, a.H, a.T, a.Hl, a.Wl, a.d = Bn, Hn, T, int(Hl), int(Wl), d
+    a.eps = float(eps)
+    a.stream = _stream(stream).value
+    check(lib().vda_prep(ctypes.byref(a)), "vda_prep")
+    return tuple(outs)
 
 
 def vda_text_state(k_text, v_text, beta_text, S_out=None, workspace=None, stream=None):

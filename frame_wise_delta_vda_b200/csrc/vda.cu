@@ -19,6 +19,7 @@
 #include "common.cuh"
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
+#include "kernels_prep.cuh"
 
 namespace {
 
@@ -331,7 +332,55 @@ int noalloc_scratch(char** out) {
 }  // namespace
 
 // ============================================================================
+namespace {
+template <int D>
+int launch_prep(const vda_prep_args& a) {
+  using namespace vda::prep;
+  cudaStream_t s = static_cast<cudaStream_t>(a.stream);
+  const size_t smem = kv_smem_bytes(a.Wl, D);
+  const float eps = a.eps > 0.f ? a.eps : 1e-6f;
+  if (cudaFuncSetAttribute(k_prep_kv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return VDA_ERR_CUDA;
+  k_prep_kv<D><<<dim3((unsigned)a.Hl, (unsigned)(a.B * a.H), 2), kThreads, smem, s>>>(
+      static_cast<const __nv_bfloat16*>(a.k_in), static_cast<const __nv_bfloat16*>(a.v_in), a.wk_s, a.wk_t, a.wv_s,
+      a.wv_t, static_cast<__nv_bfloat16*>(a.k_out), static_cast<__nv_bfloat16*>(a.v_out), a.H, a.T, a.Hl, a.Wl, eps);
+  if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  const size_t warps = (size_t)a.B * a.T * a.Hl * a.Wl * a.H;
+  const size_t blocks = (warps * 32 + 255) / 256;
+  k_prep_q<D><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.q_in),
+                                               static_cast<__nv_bfloat16*>(a.q_out), a.B, a.H, a.T,
+                                               a.Hl * a.Wl, eps);
+  if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  return VDA_OK;
+}
+}  // namespace
+
 extern "C" {
+
+int vda_prep(const vda_prep_args* a) {
+  if (!a) return VDA_ERR_INVALID_ARGUMENT;
+  if (a->B < 1 || a->H < 1 || a->T < 1 || a->Hl < 1 || a->Wl < 1 || a->d < 1) return VDA_ERR_INVALID_ARGUMENT;
+  const void* req[] = {a->q_in, a->k_in, a->v_in, a->wk_s, a->wk_t, a->wv_s, a->wv_t, a->q_out, a->k_out, a->v_out};
+  for (const void* ptr : req)
+    if (!ptr || !aligned16(ptr)) return VDA_ERR_INVALID_ARGUMENT;
+  const int d = a->d;
+  if (d != 16 && d != 32 && d != 64 && d != 128) return VDA_ERR_UNSUPPORTED;
+  const int ns = vda::prep::kThreads / (d / 2);
+  if ((a->Wl + ns - 1) / ns > vda::prep::kMaxWc) return VDA_ERR_UNSUPPORTED;
+  int dev = 0, max_smem = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return VDA_ERR_CUDA;
+  if (vda::prep::kv_smem_bytes(a->Wl, d) > (size_t)max_smem) return VDA_ERR_UNSUPPORTED;
+  if ((double)a->B * a->H * a->T * a->Hl * a->Wl * d > 4.0e12 || (double)a->B * a->H > 65535.0 || a->Hl > 2147483647)
+    return VDA_ERR_UNSUPPORTED;
+  switch (d) {
+    case 16: return launch_prep<16>(*a);
+    case 32: return launch_prep<32>(*a);
+    case 64: return launch_prep<64>(*a);
+    default: return launch_prep<128>(*a);
+  }
+}
 
 const char* vda_status_string(int status) {
   switch (status) {

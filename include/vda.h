@@ -203,6 +203,40 @@ VDA_API int vda_timing_read(float* stage_ms, int n_stages, int* calls);
  * bridge products of Eq. A.4). */
 VDA_API int vda_launches_per_forward(int B, int H, int T, int U, int d_k, int d_v, int chunk, int dtype);
 
+/* ---------------------------------------------------------------------------
+ * Feature preparation of the linear branch (Section 2.3; the fused "VDA-Prep"
+ * step of Section 5), the step ahead of vda_forward:
+ *   q' = L2(q),  k' = L2(SiLU(conv(k))),  v' = SiLU(conv(v))
+ * conv = a depthwise 5 x 5 spatial filter over the Hl x Wl latent grid then a
+ * depthwise five-tap temporal filter over the interior frames, both
+ * cross-correlations with zero padding 2 on every side; L2(x) =
+ * x / sqrt(sum(x^2) + eps) over the head dimension.
+ *   q_in, k_in, v_in  [B, T, U, H, d] bf16 (the projections of the interior
+ *                     video tokens, heads inner; token u = y * Wl + x)
+ *   wk_s, wv_s        [H, d, 5, 5] float32, wk_t, wv_t [H, d, 5] float32
+ *   q_out, k_out, v_out [B, H, T, U, d] bf16 (the layout vda_forward reads)
+ * Supported: bf16, d in {16, 32, 64, 128}, Wl * d * 20 bytes of shared
+ * memory within the device limit and at most 16 grid columns per thread
+ * slice (Wl <= 64 at d = 128).  Inputs and outputs must not overlap.
+ * Returns vda_status. */
+typedef struct vda_prep_args {
+  const void* q_in;
+  const void* k_in;
+  const void* v_in;
+  const float* wk_s;
+  const float* wk_t;
+  const float* wv_s;
+  const float* wv_t;
+  void* q_out;
+  void* k_out;
+  void* v_out;
+  int B, H, T, Hl, Wl, d;
+  float eps;                  /* L2 epsilon; <= 0 selects 1e-6 */
+  void* stream;               /* cudaStream_t */
+} vda_prep_args;
+
+VDA_API int vda_prep(const vda_prep_args* args);
+
 /* Human-readable name of a vda_status value. */
 VDA_API const char* vda_status_string(int status);
 

@@ -111,3 +111,20 @@ def test_timing_read_without_calls(L):
     calls = ctypes.c_int(-1)
     assert L.vda_timing_read(ms, 4, ctypes.byref(calls)) == 0
     assert calls.value == 0 and list(ms) == [0.0] * 4
+
+
+def test_prep_argument_checks_without_a_gpu(L):
+    """vda_prep validates its arguments before touching the device."""
+    from frame_wise_delta_vda_b200._lib import VdaPrepArgs
+    assert L.vda_prep(None) == 1
+    a = VdaPrepArgs()
+    for f in ("q_in", "k_in", "v_in", "wk_s", "wk_t", "wv_s", "wv_t", "q_out", "k_out", "v_out"):
+        setattr(a, f, 4096)            # aligned placeholders, never dereferenced
+    a.B, a.H, a.T, a.Hl, a.Wl, a.d = 1, 2, 3, 4, 5, 48
+    assert L.vda_prep(ctypes.byref(a)) == 2          # d not supported
+    a.d = 64
+    a.k_in = 4100                                     # misaligned
+    assert L.vda_prep(ctypes.byref(a)) == 1
+    a.k_in = 4096
+    a.T = 0
+    assert L.vda_prep(ctypes.byref(a)) == 1
