@@ -26,12 +26,15 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _check_tensor(name, t, dtype=None, shape=None, device=None, allow_none=False):
+def _check_tensor(name, t, dtype=None, shape=None, device=None, allow_none=False, on_host=False):
     if t is None:
         if allow_none:
             return
         raise ValueError(f"{name} is required")
-    if not t.is_cuda:
+    if on_host:
+        if t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor")
+    elif not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if device is not None and t.device != device:
         raise ValueError(f"{name} is on {t.device}, expected {device}")
@@ -54,7 +57,8 @@ def make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, windo
     if dt is None:
         raise ValueError(f"unsupported dtype {q.dtype} (bf16 or float32)")
     dev = q.device
-    chk = _check_tensor if check_device else (lambda *a, **k: None)
+    # host tensors (vda_forward_host) get the same shape and dtype checks
+    chk = _check_tensor if check_device else (lambda *a, **k: _check_tensor(*a[:4], None, **k, on_host=True))
     chk("q", q, q.dtype, (Bn, Hn, T, U, d_k), dev)
     chk("k", k, q.dtype, (Bn, Hn, T, U, d_k), dev)
     chk("v", v, q.dtype, (Bn, Hn, T, U, d_v), dev)
