@@ -80,8 +80,11 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv") \
-            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else f"/tmp/vda_clocks_{os.getpid()}.csv"
+        # the raw samples go to $VDA_CLOCKS_DIR when it names a directory (kept
+        # beside the run's other logs), else to a temporary file
+        out_dir = os.environ.get("VDA_CLOCKS_DIR", "")
+        self.path = os.path.join(out_dir, f"clocks_rank{index}.csv") if out_dir and os.path.isdir(out_dir) \
+            else f"/tmp/vda_clocks_{os.getpid()}_{index}.csv"
 
     def start(self):
         try:
