@@ -136,7 +136,7 @@ def forward_scan(S0, A_all, B_all, alpha=None):
 
 def reverse_scan(S0, A_all, B_all, alpha=None):
     """Reverse states R_t = (R_{t+1} Diag(alpha_t) + B_t)(I + A_t)^{-1},
-    R_T = S0: the same frame update taken from the last interior frame down.
+    R_T = S0: the same frame update, run backwards from frame T-1 to frame 0.
     Returns the list [R_0, ..., R_{T-1}] indexed by frame."""
     T = len(A_all)
     R = _f64(S0)
