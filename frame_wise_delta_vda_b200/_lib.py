@@ -72,6 +72,7 @@ _SIGNATURES = {
     "vda_launches_per_forward": (c_int, [c_int] * 8),
     "vda_status_string": (ctypes.c_char_p, [c_int]),
     "vda_prep": (c_int, [ctypes.POINTER(VdaPrepArgs)]),
+    "vda_selftest_wait_timeout": (c_int, [c_int, c_void_p]),
 }
 
 _lib = None

@@ -19,6 +19,23 @@ __device__ __forceinline__ void raise_device_error(unsigned int code) {
   atomicOr(&g_device_error, code);
 }
 
+// Failure-detection self test: a flag that nothing ever sets, and a kernel
+// whose single thread waits for it with the same kind of bounded poll the
+// pipelines use.  The wait runs out after max_polls polls, records a wait
+// time-out in the error word and the kernel returns normally, so the
+// context stays usable.
+__device__ int g_selftest_flag = 0;
+
+__global__ void k_wait_selftest(long long max_polls) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  volatile int* flag = &g_selftest_flag;
+  for (long long i = 0; i < max_polls; ++i) {
+    if (*flag != 0) return;
+    __nanosleep(128);
+  }
+  raise_device_error(kErrWaitTimeout);
+}
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

@@ -583,6 +583,12 @@ int vda_forward_noalloc(const vda_args* args) {
   return forward_impl(*args, scratch, p, nullptr, nullptr);
 }
 
+int vda_selftest_wait_timeout(int max_polls, void* stream) {
+  if (max_polls < 1 || max_polls > 1000000) return VDA_ERR_INVALID_ARGUMENT;
+  vda::k_wait_selftest<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((long long)max_polls);
+  return cudaGetLastError() == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+}
+
 int vda_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return VDA_ERR_CUDA;
   unsigned int word = 0, zero = 0;

@@ -189,6 +189,15 @@ VDA_API int vda_forward_noalloc(const vda_args* args);
  * bounded wait since the last call, VDA_ERR_CUDA on a CUDA error, else VDA_OK. */
 VDA_API int vda_device_status(void* stream);
 
+/* Failure-detection self test: launches one kernel that waits, with a bounded
+ * poll, on a device flag that nothing sets.  After max_polls polls (1 ..
+ * 1000000, about 0.1 us each) it gives up, records a wait time-out in the
+ * device error word and returns normally, so the context stays usable; the
+ * next vda_device_status(stream) returns VDA_ERR_TIMEOUT and clears it.
+ * No compute path calls this; it exists to test failure detection without
+ * a GPU fault.  Returns vda_status. */
+VDA_API int vda_selftest_wait_timeout(int max_polls, void* stream);
+
 /* Per-stage device timing for profiling.  vda_timing_enable(n) makes the next
  * n forward calls record CUDA events between their stages (stats, inverse,
  * scan, readout) on the call's stream; vda_timing_read(ms, 4, &calls)
