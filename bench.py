@@ -474,6 +474,7 @@ def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches):
     tokens = wl.tokens * world
     line = {
         "metric": METRIC, "value": tokens / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
+        "head_tokens_per_s": tokens * wl.H / (ms_max * 1e-3),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
