@@ -93,3 +93,27 @@ def test_binding_checks_shapes_before_the_library():
                       check_device=False)
     a = api.make_args(*args, check_device=False, alpha=z(B, H, T, d))
     assert a.alpha is not None
+
+
+def test_bench_line_carries_the_contract_keys(capsys):
+    """emit() with made-up timings prints one JSON line with the keys the
+    benchmark contract names (no GPU involved)."""
+    import json
+    import types
+    b = _bench()
+    wl = gen.WORKLOADS["full"]
+    args = types.SimpleNamespace(steps=7, warmup=3, no_cpu_baseline=True)
+    stage = {"stats": 0.35 * 7, "inverse": 0.32 * 7, "scan": 0.19 * 7, "readout": 0.40 * 7}
+    clocks = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 9}
+    e2e = {"e2e_s": 0.058, "h2d": 123, "d2h": 45}
+    b.emit(args, wl, 1, 1.3, stage, 7, clocks, e2e, 28)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "clocks", "e2e", "gpu_launches",
+              "head_tokens_per_s"):
+        assert k in line, k
+    assert line["value"] == pytest.approx(wl.tokens / 1.3e-3)
+    assert line["roofline"]["stage"] == "readout" and line["roofline"]["kernel"] == "k_readout_tc"
+    assert line["roofline"]["frac"] == pytest.approx(line["roofline"]["achieved"] / line["roofline"]["peak"])
+    assert line["e2e"]["h2d_bytes_per_step"] == 123 and line["e2e"]["d2h_bytes_per_step"] == 45
+    assert "workload" in line["config"] and line["scaling"] == "weak"
