@@ -8,6 +8,9 @@ from .vda_ref import (  # noqa: F401
     batch_rule_update,
     decayed,
     boundary_states,
+    boundary_states_by_chunk_maps,
+    compose_maps,
+    frame_map,
     frame_stats,
     frame_update,
     forward_scan,

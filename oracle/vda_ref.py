@@ -249,6 +249,49 @@ def boundary_states(P, R, S0_fwd, S0_rev, T, chunk):
     return np.stack([np.stack(fwd), np.stack(rev)])
 
 
+def frame_map(A, B, alpha_t=None):
+    """The frame update as an affine map of the entering state (Appendix A.1,
+    Eq. A.1): S_t = S_{t-1} M_t + J_t with M_t = Diag(alpha_t)(I + A_t)^{-1}
+    and J_t = B_t (I + A_t)^{-1}.  Returns (M_t, J_t)."""
+    A = _f64(A)
+    d_k = A.shape[0]
+    inv = np.linalg.inv(np.eye(d_k) + A)
+    M = inv if alpha_t is None else _f64(alpha_t)[:, None] * inv
+    return M, _f64(B) @ inv
+
+
+def compose_maps(first, second):
+    """Apply `first` then `second`: S -> (S M1 + J1) M2 + J2 = S (M1 M2) + (J1 M2 + J2)."""
+    (M1, J1), (M2, J2) = first, second
+    return M1 @ M2, J1 @ M2 + J2
+
+
+def boundary_states_by_chunk_maps(A_all, B_all, S0_fwd, S0_rev, T, chunk, alpha=None):
+    """A second route to the boundary states (the chunk-wise scan of Section 5):
+    each chunk's frames are composed into one affine map (Eq. A.1), in frame
+    order for the forward scan and in reverse frame order for the reverse scan,
+    and the short chunk sequence is scanned in both directions.  Returns the
+    same [2, NC+1, d_v, d_k] array as boundary_states."""
+    nc = num_chunks(T, chunk)
+    maps = [frame_map(A_all[t], B_all[t], None if alpha is None else alpha[t]) for t in range(T)]
+    fwd = [_f64(S0_fwd)]
+    for j in range(nc):
+        frames = range(j * chunk, min(T, (j + 1) * chunk))
+        m = None
+        for t in frames:
+            m = maps[t] if m is None else compose_maps(m, maps[t])
+        fwd.append(fwd[-1] @ m[0] + m[1])
+    rev = [None] * (nc + 1)
+    rev[nc] = _f64(S0_rev)
+    for j in range(nc - 1, -1, -1):
+        frames = range(min(T, (j + 1) * chunk) - 1, j * chunk - 1, -1)
+        m = None
+        for t in frames:
+            m = maps[t] if m is None else compose_maps(m, maps[t])
+        rev[j] = rev[j + 1] @ m[0] + m[1]
+    return np.stack([np.stack(fwd), np.stack(rev)])
+
+
 def vda_forward(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev,
                 chunk, window_chunks, eps=RMS_EPS, heads=None, alpha=None):
     """Whole-tensor wrapper: q, k: [B, H, T, U, d_k]; v, gate: [B, H, T, U, d_v];

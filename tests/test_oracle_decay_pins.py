@@ -130,3 +130,17 @@ def test_scalar_decay_keeps_rotation_invariance():
     y_rot = ref.vda_forward_head(q @ Rm.T, k @ Rm.T, v, beta, g, wt, S0f @ Rm.T, S0r @ Rm.T, C, w,
                                  alpha=alpha)
     np.testing.assert_allclose(y_rot, y, atol=1e-12)
+
+
+@pytest.mark.parametrize("T,C,decay", [(10, 5, False), (11, 4, True), (7, 3, True), (6, 1, False), (5, 5, True)])
+def test_chunk_composed_maps_give_the_boundary_states(T, C, decay):
+    """Eq. A.1's affine form composed chunk by chunk (the chunk-wise scan of
+    Section 5) reaches the same boundary states as the frame-by-frame scans,
+    in both directions, with and without decay."""
+    rng = np.random.default_rng(600 + 10 * T + C)
+    q, k, v, beta, g, wt, S0f, S0r, alpha = _case(rng, T)
+    a = alpha if decay else None
+    _, inter = ref.vda_forward_head(q, k, v, beta, g, wt, S0f, S0r, C, 1, keep=True, alpha=a)
+    want = ref.boundary_states(inter["P"], inter["R"], S0f, S0r, T, C)
+    got = ref.boundary_states_by_chunk_maps(inter["A"], inter["B"], S0f, S0r, T, C, alpha=a)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-11)
