@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=None,
                     help="timed steps of the host-buffer (end-to-end) measurement; 0 skips it")
-    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(gen.WORKLOADS),
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(gen.WORKLOADS) + sorted(gen.PREP_WORKLOADS),
                     help="workload to run (the benchmark line is defined on 'full'; other "
                          "workloads serve profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -217,6 +217,8 @@ def run_reference(args):
     if rank != 0:
         return
     import oracle as ref
+    if args.workload not in gen.WORKLOADS:
+        raise SystemExit(f"{args.workload} is a feature-preparation workload; the reference arm times the forward")
     wl = gen.WORKLOADS[args.workload]
     x = gen.head_inputs(wl, 0, 0)
     w = gen.rms_weight(wl)
@@ -264,7 +266,7 @@ def run_prep(args):
     from frame_wise_delta_vda_b200 import api
     from frame_wise_delta_vda_b200._lib import lib
     lib()
-    pw = gen.PREP_WORKLOADS["prep_full"]
+    pw = gen.PREP_WORKLOADS[args.workload if args.workload in gen.PREP_WORKLOADS else "prep_full"]
     x = gen.make_prep_inputs(pw)
 
     def dev_t(a):
@@ -343,6 +345,8 @@ def main():
     from frame_wise_delta_vda_b200._lib import lib
     lib()  # fail loudly without the CUDA library
 
+    if args.workload not in gen.WORKLOADS:
+        raise SystemExit(f"{args.workload} is a feature-preparation workload: use --prep")
     base = gen.WORKLOADS[args.workload]
     # every rank runs its own problem of the same size (weak scaling)
     wl = gen.Workload(**{**base.__dict__, "seed": ranks.rank_seed(base.seed, rank)})

@@ -217,6 +217,8 @@ class PrepWorkload:
 PREP_WORKLOADS = {
     "prep_small": PrepWorkload("prep_small", 1, 4, 6, 6, 8, 64, 21),
     "prep_odd": PrepWorkload("prep_odd", 2, 3, 5, 3, 7, 128, 22),
+    # the full-size grid with 16 heads and 20 frames (0.25 GB per direction): profiling size
+    "prep_mid": PrepWorkload("prep_mid", 1, 16, 20, 24, 42, 128, 24),
     # the full-size shapes: 60 interior frames of a 24 x 42 latent grid
     "prep_full": PrepWorkload("prep_full", 1, 48, 60, 24, 42, 128, 23),
 }
