@@ -8,7 +8,8 @@ float64 oracle can consume the same inputs without sharing any code.
 The five workloads follow the paper's 14.3 s, 768p setting in shape
 (latent video (24, 102, 48, 84) -> 100 interior frames, 24 x 42 = 1008 tokens
 per frame after 2 x 2 patchify, chunk = 5 latent frames, window = own chunk
-+-1) at reduced and full scale; see the design notes for the recipe.
++-1) at reduced and full scale; each workload's shapes, distributions and
+seed are stated in its `Workload` entry below.
 
 Every (tensor, batch, head) stream has its own numpy SeedSequence
 (entropy = [seed, tensor id, b, h]), so any head can be regenerated alone

@@ -10,7 +10,7 @@ convolution to K and V, a depthwise 5 x 5 spatial filter and a five-tap
 temporal filter, then SiLU; Q and K are L2-normalised; the result is laid
 out frame-major per head.
 
-Readings of what the pages leave open (each is listed in the design notes):
+Readings of what the pages leave open:
   * inputs are the projections of the interior video tokens, [B, T, U, H, d]
     (frame-major tokens, heads inner), token u = y * Wl + x on the Hl x Wl
     latent grid; outputs are [B, H, T, U, d];

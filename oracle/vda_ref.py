@@ -14,7 +14,7 @@ Notation (per batch b, head h, interior latent frame t):
   K_t in R^{U x d_k}, V_t in R^{U x d_v}, beta_t in R^U, Q_t in R^{U x d_k},
   G_t in R^{U x d_v} (gate logits), state S in R^{d_v x d_k}, read as o = S q.
 
-Readings of points the paper leaves open (each is listed in the design notes):
+Readings of points the paper leaves open:
   * decay: without `alpha` the gate is 1, so S_bar_t = S_{t-1} and there is no
     decay bridge; with `alpha` [T, d_k] in [0, 1] (Eq. 2) both scans use
     S_bar_t = S_{t+-1} Diag(alpha_t) with the frame's own alpha_t, and query

@@ -10,12 +10,13 @@ from frame_wise_delta_vda_b200 import inputs as gen
 
 # output tolerance per I/O dtype (relative Frobenius error per (b, h))
 TOL = {"bf16": 1e-2, "f32": 1e-4}
-# diagnostic bound for intermediates (A, B, M, boundary states).  float32 I/O:
-# 10x tighter than the output bound.  bf16 I/O: A is built from beta*K rounded
-# to bf16 (relative error up to 2^-9 per product, a measured design choice
-# whose cost at the output is about 2e-3 on the correlated-key workload), and
-# M and the states inherit that, so the bound is half the output bound.
-TOL_INTER = {"bf16": 5e-3, "f32": 1e-5}
+# diagnostic bound for intermediates (A, B, M, boundary states): 10x tighter
+# than the output bound for both I/O dtypes.  On the bf16 path the Gram
+# builder splits beta*K into bf16 hi + lo and the inverse, scan and readout
+# feed the tensor cores hi/lo operand pairs (about 16 significant bits,
+# fp32 accumulation), so the intermediates keep roughly 1e-4 relative
+# accuracy even on the correlated-key stress workload.
+TOL_INTER = {"bf16": 1e-3, "f32": 1e-5}
 
 
 def to_torch(arr, device):

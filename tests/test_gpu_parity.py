@@ -2,8 +2,7 @@
 
 Bar: relative Frobenius error per (b, h) <= 1e-2 for bf16 I/O and <= 1e-4 for
 float32 I/O; intermediates (A, B, M, boundary states) are diagnostic, with
-the bounds of TOL_INTER (10x tighter for float32, half the output bound for
-bf16).  Full-size workloads run in the launch configuration the
+the bounds of TOL_INTER (10x tighter than the output bound).  Full-size workloads run in the launch configuration the
 benchmark times and are compared on sampled heads.
 """
 
@@ -62,21 +61,22 @@ def test_workload_parity_all_heads(name):
     y = to_numpy_f64(out)
     st = states.cpu().double().numpy()
     sa = stats.cpu().double().numpy()
-    worst = 0.0
+    worst = {"out": 0.0, "states": 0.0, "A": 0.0, "B": 0.0, "M": 0.0}
     for b in range(wl.B):
         for h in range(wl.H):
             xh = _head_x(x, b, h)
             y_ref, inter = oracle_head(xh, wl, keep=True)
             e = rel_err(y[b, h], y_ref)
-            worst = max(worst, e)
+            worst["out"] = max(worst["out"], e)
             assert e <= TOL[wl.dtype], (name, b, h, e)
             bs = ref.boundary_states(inter["P"], inter["R"], np.zeros((wl.d, wl.d)),
                                      np.zeros((wl.d, wl.d)), wl.T, wl.chunk)
-            assert rel_err(st[:, b, h], bs) <= TOL_INTER[wl.dtype], ("states", b, h)
-            assert rel_err(sa[0, b, h], inter["A"]) <= TOL_INTER[wl.dtype], ("A", b, h)
-            assert rel_err(sa[1, b, h], inter["B"]) <= TOL_INTER[wl.dtype], ("B", b, h)
-            assert rel_err(sa[2, b, h], inter["M"]) <= TOL_INTER[wl.dtype], ("M", b, h)
-    print(f"{name}: worst per-head rel err {worst:.3e}")
+            errs = {"states": rel_err(st[:, b, h], bs), "A": rel_err(sa[0, b, h], inter["A"]),
+                    "B": rel_err(sa[1, b, h], inter["B"]), "M": rel_err(sa[2, b, h], inter["M"])}
+            for key, e in errs.items():
+                worst[key] = max(worst[key], e)
+                assert e <= TOL_INTER[wl.dtype], (key, b, h, e)
+    print(f"{name}: worst per-head rel err " + ", ".join(f"{k} {v:.3e}" for k, v in worst.items()))
 
 
 def test_tiny_output_is_exactly_zero():

@@ -40,6 +40,9 @@ def test_stage_kernels_follow_the_path():
     b = _bench()
     tc = b.stage_kernels(gen.WORKLOADS["full"])
     assert tc["readout"][1] == "k_readout_tc" and tc["inverse"][1] == "k_inverse_tc"
+    # the streaming kernels are HBM-limited; the inverse and the scan are dependent chains
+    assert tc["stats"][0] == tc["readout"][0] == "hbm"
+    assert tc["inverse"][0] == tc["scan"][0] == "latency"
     simt = b.stage_kernels(gen.WORKLOADS["tiny"])
     assert simt["readout"][1] == "k_readout_simt" and simt["inverse"] == ("alu", "k_gj_inverse", ["kernels_simt.cuh"])
 
