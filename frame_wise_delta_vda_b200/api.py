@@ -212,10 +212,11 @@ def vda_forward_noalloc(q, k, v, beta, gate, rms_weight, S0_fwd=None, S0_rev=Non
                         window_chunks=1, out=None, eps=1e-6, stream=None, alpha=None):
     """Forward through `vda_forward_noalloc`: the library uses its fixed
     internal scratch array instead of any allocation (sizes must fit in
-    NOALLOC_SCRATCH_BYTES of workspace).  `out` must be preallocated by callers
-    that cannot allocate; it is created here only as a convenience."""
+    NOALLOC_SCRATCH_BYTES of workspace).  The caller passes a preallocated
+    `out`: this route exists for callers that cannot allocate, so it never
+    creates a tensor itself."""
     if out is None:
-        out = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
+        raise ValueError("vda_forward_noalloc needs a preallocated `out` (this route allocates nothing)")
     a = make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks, eps, stream,
                   alpha=alpha)
     check(lib().vda_forward_noalloc(ctypes.byref(a)), "vda_forward_noalloc")

@@ -77,6 +77,7 @@ struct Timing {
   int max_calls = 0;
   int calls = 0;
   std::vector<cudaEvent_t> ev;  // (kStages + 1) per call
+  std::vector<char> done;       // 1 once every event of the call's slot was recorded
 } g_timing;
 
 void timing_mark(int call_slot, int stage, cudaStream_t s) {
@@ -88,6 +89,22 @@ int timing_begin_call() {
   std::lock_guard<std::mutex> lk(g_timing.mu);
   if (g_timing.max_calls <= 0 || g_timing.calls >= g_timing.max_calls) return -1;
   return g_timing.calls++;
+}
+
+// a forward that returns early leaves its slot incomplete: vda_timing_read skips it
+void timing_end_call(int call_slot) {
+  if (call_slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_timing.mu);
+  g_timing.done[(size_t)call_slot] = 1;
+}
+
+void timing_reset_locked() {
+  for (cudaEvent_t e : g_timing.ev)
+    if (e) cudaEventDestroy(e);
+  g_timing.ev.clear();
+  g_timing.done.clear();
+  g_timing.calls = 0;
+  g_timing.max_calls = 0;
 }
 
 // ----------------------------------------------------------------------------
@@ -192,6 +209,7 @@ int forward_impl(const vda_args& a, char* ws, const Plan& p, float* states_out, 
     rc = dispatch_simt<float>(p, a, ws, s, tslot, stats_out);
   }
   if (rc != VDA_OK) return rc;
+  timing_end_call(tslot);
   if (states_out) {
     const size_t bytes = 2 * p.BH * (size_t)(p.NC + 1) * p.d * p.d * sizeof(float);
     if (cudaMemcpyAsync(states_out, ws + p.off_states, bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
@@ -309,23 +327,14 @@ HostLayout host_layout(int B, int H, int T, int U, int d, int chunk, int dtype) 
 // cudaGetSymbolAddress (the symbol itself is a host-side stand-in).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[VDA_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {};
-
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device (with that device current) and cached.
+// Device address of g_noalloc_scratch in the current context.  Looked up on
+// every call (the lookup allocates nothing): an address cached per device
+// number would go stale after cudaDeviceReset, or belong to another context
+// when a host runs the library under a non-primary context.
 int noalloc_scratch(char** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return VDA_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return VDA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
-      return VDA_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = static_cast<char*>(g_noalloc_ptr[dev]);
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return VDA_ERR_CUDA;
+  *out = static_cast<char*>(ptr);
   return VDA_OK;
 }
 
@@ -516,6 +525,9 @@ int vda_forward_host(const vda_args* ha, void* device_buffer, size_t device_byte
   const size_t per_head_tok = (size_t)ha->T * ha->U;
   const int d = ha->d_k;
 #define VDA_CK(x) do { if ((x) != cudaSuccess) return VDA_ERR_CUDA; } while (0)
+  // the copy / compute pipeline; on an error it returns at once, with copies
+  // possibly still queued on the three streams
+  auto run_groups = [&]() -> int {
   VDA_CK(cudaMemcpyAsync(d_w, ha->rms_weight, L.sz_w, cudaMemcpyHostToDevice, P->h2d));
   for (int g = 0; g < L.groups; ++g) {
     const int sl = g & 1;
@@ -556,8 +568,8 @@ int vda_forward_host(const vda_args* ha, void* device_buffer, size_t device_byte
     a.out = S + L.slot_off_out;
     a.stream = P->comp;
     const Plan p = make_plan(1, nh, a.T, a.U, d, a.chunk, a.window_chunks, a.dtype);
-    rc = forward_impl(a, S + L.slot_off_ws, p, nullptr, nullptr);
-    if (rc != VDA_OK) return rc;
+    const int frc = forward_impl(a, S + L.slot_off_ws, p, nullptr, nullptr);
+    if (frc != VDA_OK) return frc;
     VDA_CK(cudaEventRecord(P->comp_done[sl], P->comp));
 
     VDA_CK(cudaStreamWaitEvent(P->d2h, P->comp_done[sl], 0));
@@ -567,8 +579,19 @@ int vda_forward_host(const vda_args* ha, void* device_buffer, size_t device_byte
   }
   VDA_CK(cudaStreamSynchronize(P->d2h));
   VDA_CK(cudaStreamSynchronize(P->comp));
-#undef VDA_CK
   return VDA_OK;
+  };
+#undef VDA_CK
+  rc = run_groups();
+  if (rc != VDA_OK) {
+    // the call is synchronous: no queued copy may read or write the caller's
+    // host buffers after it returns, so drain every stream (their status is
+    // not needed: the first error is the one reported)
+    cudaStreamSynchronize(P->h2d);
+    cudaStreamSynchronize(P->comp);
+    cudaStreamSynchronize(P->d2h);
+  }
+  return rc;
 }
 
 int vda_forward_noalloc(const vda_args* args) {
@@ -602,14 +625,15 @@ int vda_device_status(void* stream) {
 
 int vda_timing_enable(int max_calls) {
   std::lock_guard<std::mutex> lk(g_timing.mu);
-  for (cudaEvent_t e : g_timing.ev) cudaEventDestroy(e);
-  g_timing.ev.clear();
-  g_timing.calls = 0;
-  g_timing.max_calls = 0;
+  timing_reset_locked();
   if (max_calls <= 0) return VDA_OK;
-  g_timing.ev.resize((size_t)max_calls * (kStages + 1));
+  g_timing.ev.assign((size_t)max_calls * (kStages + 1), nullptr);
+  g_timing.done.assign((size_t)max_calls, 0);
   for (auto& e : g_timing.ev)
-    if (cudaEventCreate(&e) != cudaSuccess) return VDA_ERR_CUDA;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      timing_reset_locked();
+      return VDA_ERR_CUDA;
+    }
   g_timing.max_calls = max_calls;
   return VDA_OK;
 }
@@ -618,22 +642,22 @@ int vda_timing_read(float* stage_ms, int n_stages, int* calls) {
   std::lock_guard<std::mutex> lk(g_timing.mu);
   if (!stage_ms || n_stages < 1) return VDA_ERR_INVALID_ARGUMENT;
   for (int i = 0; i < n_stages; ++i) stage_ms[i] = 0.f;
-  const int n = g_timing.calls;
-  for (int c = 0; c < n; ++c) {
+  int rc = VDA_OK, complete = 0;
+  for (int c = 0; c < g_timing.calls && rc == VDA_OK; ++c) {
+    if (!g_timing.done[(size_t)c]) continue;   // a forward that failed part-way
     cudaEvent_t* e = &g_timing.ev[(size_t)c * (kStages + 1)];
-    if (cudaEventSynchronize(e[kStages]) != cudaSuccess) return VDA_ERR_CUDA;
+    if (cudaEventSynchronize(e[kStages]) != cudaSuccess) { rc = VDA_ERR_CUDA; break; }
     for (int st = 0; st < std::min(n_stages, kStages); ++st) {
       float ms = 0.f;
-      if (cudaEventElapsedTime(&ms, e[st], e[st + 1]) != cudaSuccess) return VDA_ERR_CUDA;
+      if (cudaEventElapsedTime(&ms, e[st], e[st + 1]) != cudaSuccess) { rc = VDA_ERR_CUDA; break; }
       stage_ms[st] += ms;
     }
+    ++complete;
   }
-  if (calls) *calls = n;
-  for (cudaEvent_t e : g_timing.ev) cudaEventDestroy(e);
-  g_timing.ev.clear();
-  g_timing.calls = 0;
-  g_timing.max_calls = 0;
-  return VDA_OK;
+  if (calls) *calls = complete;
+  // events are released and timing is switched off whatever happened above
+  timing_reset_locked();
+  return rc;
 }
 
 }  // extern "C"

@@ -172,9 +172,11 @@ VDA_API int vda_forward_host(const vda_args* host_args, void* device_buffer, siz
  * which every GPU that loads the library holds until the process exits.
  *   - Returns VDA_ERR_WORKSPACE when the sizes need more scratch than that
  *     (vda_workspace_bytes() > VDA_NOALLOC_SCRATCH_BYTES); nothing is launched.
- *   - The first call on each device looks up the array's device address with
- *     the CUDA runtime (no allocation); make that first call before any stream
- *     capture begins.
+ *   - Every call looks up the array's device address in the current context
+ *     with the CUDA runtime (cudaGetSymbolAddress; no allocation), so the
+ *     address is never stale after cudaDeviceReset or under another context.
+ *     The first lookup in a context may load the library's device code; make
+ *     the first call on each device before any stream capture begins.
  *   - Calls share the one array: two calls whose work overlaps on the GPU
  *     (different streams, or different host threads, without ordering between
  *     them) race and corrupt each other's results.  Every scratch word is
