@@ -316,39 +316,51 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
 
 // ===========================================================================
 // k_inverse_tc: M = (I + A)^{-1} for every frame-head, by a block sweep of the
-// symmetric positive definite I + A held in TMEM, with the rank-16 updates
-// on the tensor cores.  Sweeping every index of a symmetric matrix ends at
-// its negative inverse; with pivot blocks P of 16 indices, one block step
-//   G = -P^{-1}                 (16 x 16 sweep in one warp)
-//   A_ij += (C G)_i C_j^T       (i, j outside P; C = A[:, P]; one MMA)
-//   A_iP = W_i = -(C G)_i,  A_PP = G,  A_Pj = W_j^T   (fix-ups)
-// sweeps the 16 indices of P at once.  Every pivot block of an SPD matrix's
-// Schur complement is SPD, so no pivoting is needed.  C G is formed on the
-// CUDA cores in fp32; C and C G go to the tensor cores as bf16 hi + lo (three
-// products, ~16 significant bits).  The 16 x 16 sweep is the sequential part,
-// so it runs one block ahead: while the tensor cores update the matrix with
-// block P, the warp owning the next block Q brings A_QQ up to date itself
-// (A_QQ + (C G)_Q C_Q^T in fp32) and sweeps it.  Four warpgroups per CTA
-// work on four matrices at once (own TMEM columns, shared-memory workspace,
-// named barrier and completion barrier).  In: A rows (fp32, from
-// k_stats_tc).  Out: the scan's M operand image (element (j, k) = M[k][j],
-// MN-major, 128-B swizzle, bf16 hi / lo halves) and optionally M in fp32.
+// symmetric positive definite I + A held in TMEM, with every product on the
+// tensor cores.  Sweeping every index of a symmetric matrix ends at its
+// negative inverse.  Sweeping a pivot block P of 16 indices, with
+// C = (I + A)[:, P] and G = -P^{-1}, maps
+//   A_ij -> A_ij + (C G)_i C_j^T   (i, j outside P; the Schur complement)
+//   A_iP -> -(C G)_i,   A_PP -> G,   A_Pj -> -(C G)_j^T.
+// TMEM holds T = the current matrix minus the identity on the indices not
+// swept yet.  One block step:
+//   1. Y = the panel T[:, P] with its P rows replaced by -e_i (then C G = Y G
+//      outside P, and -G on P);  X = Y G by MMA into T's P columns.
+//   2. T's P rows and P columns are cleared (TMEM stores), then by MMA
+//      T += X Y^T  (Schur complement outside P; -X in the P columns;
+//                   -G C_j^T in the P rows; G in the P block).
+// No term cancels in floating point: every entry is a sum of products of the
+// size of the result.  Operands go to the tensor cores as bf16 splits in three
+// parts (h, m, l; bf16 x 3 holds an fp32 value exactly): X = Y G and the
+// update X Y^T each take the six products down to 2^-24 (hh, hm, mh, hl, lh,
+// mm).  This keeps the swept matrix symmetric to ~1e-5; with fewer products
+// the asymmetry between the P rows and the P columns compounds through the
+// scan.  Every pivot block of an SPD matrix's Schur complement is SPD, so no
+// pivoting is needed.
+// The 16 x 16 sweep that gives G is the sequential part, so it runs one block
+// ahead: once X is known, the warp owning the next block Q brings A_QQ up to
+// date in fp32 (A_QQ + X_Q C_Q^T) and sweeps it while the tensor cores apply
+// the update.  Four warpgroups per CTA work on four matrices at once (own
+// TMEM columns, shared-memory workspace, named barriers, completion barriers).
+// In: A rows (fp32, from k_stats_tc).  Out: the scan's M operand image
+// (element (j, k) = M[k][j], MN-major, 128-B swizzle, bf16 hi / lo halves)
+// and optionally M in fp32.
 // ===========================================================================
 struct InvCfg {
   static constexpr int GROUPS = 4;
   static constexpr int THREADS = 128 * GROUPS;
-  static constexpr uint32_t TCOLS = 128;     // TMEM columns per group: the matrix
-  static constexpr uint32_t SW_BYTES = 28672; // per-group workspace (see SW_* below)
+  static constexpr uint32_t TCOLS = 128;      // TMEM columns per group: the matrix
+  static constexpr uint32_t SW_BYTES = 30720;  // per-group workspace (see SW_* below)
   static constexpr uint32_t BAR_OFF = GROUPS * SW_BYTES;
-  static constexpr size_t SMEM = BAR_OFF + GROUPS * 8 + 16 + 1024;
+  static constexpr int NBAR = 2 * GROUPS;      // per group: update done, X done
+  static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
 };
-// per-group workspace: K-major no-swizzle operand images (rows of 16 bf16)
-// and fp32 exchange buffers
-constexpr uint32_t SW_CH = 0, SW_CL = 4096;        // panel C, 128 rows
-constexpr uint32_t SW_CGH = 8192, SW_CGL = 12288;  // C G, 128 rows
-constexpr uint32_t SW_W = 16384;                   // W^T = (-C G)^T, [16][128]
-constexpr uint32_t SW_G = 24576;                   // G = -P^{-1}, [2 buffers][16][16]
-constexpr uint32_t SW_CQ = 26624;                  // next block's rows of C, transposed, [2 segments][16][16]
+// per-group workspace: K-major no-swizzle operand images (rows of 16 bf16,
+// 4 KB for 128 rows, 512 B for 16) and the fp32 exchange buffer
+constexpr uint32_t SW_YH = 0, SW_YM = 4096, SW_YL = 8192;         // Y in three parts (P rows: -e, 0, 0)
+constexpr uint32_t SW_XH = 12288, SW_XM = 16384, SW_XL = 20480;   // X in three parts
+constexpr uint32_t SW_GI = 24576;                                 // G in three parts, 3 x 512 B
+constexpr uint32_t SW_CQ = 26624;   // next block's rows of C, transposed, [2 steps][2 segments][16][16]
 
 // Pivot block swept at step s by group grp: the order 0,2,4,6,1,3,5,7 rotated
 // by grp.  The sweep's result does not depend on the order; this one puts
@@ -392,24 +404,79 @@ __device__ __forceinline__ void sweep16(const float (&x)[16], int sel, int lane,
   }
 }
 
-__device__ __forceinline__ void st_row8_f32(uint32_t addr, const float (&x)[8]) {
-#pragma unroll
-  for (int t = 0; t < 8; t += 4)
-    st_shared_v4(addr + 4u * t, make_uint4(__float_as_uint(x[t]), __float_as_uint(x[t + 1]),
-                                           __float_as_uint(x[t + 2]), __float_as_uint(x[t + 3])));
+// x = h + m + l exactly with bf16 h = rn(x), m = rn(x - h), l = x - h - m
+// (24 significant bits in three 8-bit parts; exact for normal values).
+__device__ __forceinline__ void split3_bf16(float x, float& h, float& m, float& l) {
+  h = __bfloat162float(__float2bfloat16_rn(x));
+  const float r = x - h;
+  m = __bfloat162float(__float2bfloat16_rn(r));
+  l = r - m;
 }
 
+// 16 fp32 values -> rows r of three no-swizzle K-major images (parts h, m, l)
+__device__ __forceinline__ void store_row16_split3(uint32_t ih, uint32_t im, uint32_t il, uint32_t r,
+                                                   const float (&x)[16]) {
+#pragma unroll
+  for (int kc = 0; kc < 2; ++kc) {
+    uint32_t hw[4], mw[4], lw[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float h0, m0, l0, h1, m1, l1;
+      split3_bf16(x[8 * kc + 2 * q], h0, m0, l0);
+      split3_bf16(x[8 * kc + 2 * q + 1], h1, m1, l1);
+      hw[q] = pack_bf16(h0, h1);
+      mw[q] = pack_bf16(m0, m1);
+      lw[q] = pack_bf16(l0, l1);
+    }
+    const uint32_t off = kimg16(r, 8u * kc);
+    st_shared_v4(ih + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+    st_shared_v4(im + off, make_uint4(mw[0], mw[1], mw[2], mw[3]));
+    st_shared_v4(il + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+  }
+}
+
+// G image (the X product's B operand): lane (r, h) of the sweeping warp holds
+// row r, columns [8h, 8h + 8) of G; three K-major no-swizzle parts h, m, l
+__device__ __forceinline__ void store_g_image(uint32_t swb, int r, int h, const float (&gq)[8]) {
+  uint32_t hw[4], mw[4], lw[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float h0, m0, l0, h1, m1, l1;
+    split3_bf16(gq[2 * q], h0, m0, l0);
+    split3_bf16(gq[2 * q + 1], h1, m1, l1);
+    hw[q] = pack_bf16(h0, h1);
+    mw[q] = pack_bf16(m0, m1);
+    lw[q] = pack_bf16(l0, l1);
+  }
+  const uint32_t off = kimg16((uint32_t)r, 8u * (uint32_t)h);
+  st_shared_v4(swb + SW_GI + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
+  st_shared_v4(swb + SW_GI + 512u + off, make_uint4(mw[0], mw[1], mw[2], mw[3]));
+  st_shared_v4(swb + SW_GI + 1024u + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+}
+
+// Barriers of one group (ids distinct per group): `bY` closes the Y images and
+// the G images of a step, `bX` the X images and the cleared rows and columns
+// of P.  The group's MMAs are issued by lane 0 of its warp grp, so the four
+// groups' issuers sit on different SM sub-partitions; that warp waits at the
+// barriers, the other warps only arrive, and each of their next arrivals
+// follows a wait on the MMA that the barrier released.
+struct InvBars {
+  uint32_t bY, bX, sbar, xbar;
+};
+
 // One warpgroup sweeps the matrix in TMEM columns [tA, tA + 128); thread i =
-// TMEM lane i; gw = warp index within the group, grp = group index.  bid:
-// the group's named barrier; bend: a second one that closes each step, so a
-// warp that only arrives at bid cannot reach bid again before every thread
-// has passed it.  Returns false on abort.
-__device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t lb, uint32_t swb, uint32_t bid,
-                                                   uint32_t bend, uint32_t sbar, uint32_t& sweep_phase,
-                                                   volatile int* abort_flag, int i, int gw, int lane, int grp) {
+// TMEM lane i; gw = warp index within the group, grp = group index.  Returns
+// false if a wait gave up (the matrix is then garbage; the barrier sequence is
+// still kept, so the group stays in step).
+__device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t lb, uint32_t swb, const InvBars& bar,
+                                                   uint32_t& sphase, uint32_t& xphase, volatile int* abort_flag,
+                                                   int i, int gw, int lane, int grp) {
   constexpr uint32_t kId128 = idesc_bf16(128, 128, 0, 0);
+  constexpr uint32_t kId16 = idesc_bf16(128, 16, 0, 0);
   const int r = lane & 15, h = lane >> 4;
-  const uint32_t cqb = swb + SW_CQ + (uint32_t)h * 1024u;
+  const bool issuer_warp = gw == grp;
+  const bool issuer = issuer_warp && lane == 0;
+  bool ok = true;
   // G of the first pivot block (the matrix is untouched: P = its own block)
   {
     const int K0 = inv_block(0, grp);
@@ -422,9 +489,8 @@ __device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t lb, uin
 #pragma unroll
       for (int t = 0; t < 16; ++t) x0[t] = __uint_as_float(v[t]) + ((in0 && r == t) ? 1.f : 0.f);
       sweep16(x0, K0 & 1, lane, g0);
-      st_row8_f32(swb + SW_G + 64u * (uint32_t)r + 32u * (uint32_t)h, g0);
+      store_g_image(swb, r, h, g0);
     }
-    named_bar_sync(bid, 128);
   }
 #pragma unroll 1
   for (int s = 0; s < 8; ++s) {
@@ -435,10 +501,16 @@ __device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t lb, uin
     const int Kn = inv_block(s + 1, grp);
     const bool qwarp = s < 7 && gw == (Kn >> 1);     // sweeps the next block ahead
     const bool inQ = qwarp && (i >> 4) == Kn;
-    const uint32_t gcur = swb + SW_G + 1024u * (uint32_t)(s & 1);
-    const uint32_t gnext = swb + SW_G + 1024u * (uint32_t)((s + 1) & 1);
-    // panel C (identity on P's diagonal); the next block's columns for its warp
-    float c[16], aq[16];
+    // by step parity: the sweeping warp of step s + 2 writes it only after
+    // passing the X barrier of step s + 1, i.e. after this step's lookahead
+    const uint32_t cqb = swb + SW_CQ + 2048u * (uint32_t)(s & 1) + 1024u * (uint32_t)h;
+    if (s > 0) {   // the previous step's update is in TMEM, its operand images are free
+      ok = mbar_wait(bar.sbar, sphase, abort_flag) && ok;
+      sphase ^= 1u;
+      tc_fence_after();
+    }
+    // raw panel T[:, P]; the next block's columns for its warp
+    float yr[16], aq[16];
     {
       uint32_t v[16];
       tmem_ld16(lb + tA + p0, v);
@@ -452,112 +524,113 @@ __device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t lb, uin
         tmem_wait_ld();
       }
 #pragma unroll
-      for (int t = 0; t < 16; ++t) c[t] = __uint_as_float(v[t]) + ((inP && r == t) ? 1.f : 0.f);
+      for (int t = 0; t < 16; ++t) yr[t] = __uint_as_float(v[t]);
     }
-    // C G in fp32 (G symmetric, broadcast from shared memory)
-    float cg[16];
+    {   // Y (P rows -e) in three parts
+      float ye[16];
 #pragma unroll
-    for (int t = 0; t < 16; ++t) cg[t] = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-#pragma unroll
-      for (int t = 0; t < 16; t += 4) {
-        const float4 x = ld_shared_f4(gcur + 64u * (uint32_t)k + 4u * t);
-        cg[t] = fmaf(c[k], x.x, cg[t]); cg[t + 1] = fmaf(c[k], x.y, cg[t + 1]);
-        cg[t + 2] = fmaf(c[k], x.z, cg[t + 2]); cg[t + 3] = fmaf(c[k], x.w, cg[t + 3]);
-      }
+      for (int t = 0; t < 16; ++t) ye[t] = inP ? (r == t ? -1.f : 0.f) : yr[t];
+      store_row16_split3(swb + SW_YH, swb + SW_YM, swb + SW_YL, (uint32_t)i, ye);
     }
-    store_row16_hilo(swb + SW_CH, swb + SW_CL, (uint32_t)i, c);
-    store_row16_hilo(swb + SW_CGH, swb + SW_CGL, (uint32_t)i, cg);
+    if (qwarp) {   // C's rows of the next block, transposed: cq[k][r] = C[Q_r][k] (Q is outside P)
 #pragma unroll
-    for (int t = 0; t < 16; ++t)   // W^T[t][i] = -(C G)[i][t]; lanes write consecutive words
-      st_shared_f1(swb + SW_W + (uint32_t)t * 512u + 4u * (uint32_t)i, -cg[t]);
-    if (qwarp) {   // C's rows of the next block, transposed: cq[k][r] = C[Q_r][k]
-#pragma unroll
-      for (int k = 0; k < 16; ++k) st_shared_f1(cqb + 64u * (uint32_t)k + 4u * (uint32_t)r, c[k]);
+      for (int k = 0; k < 16; ++k) st_shared_f1(cqb + 64u * (uint32_t)k + 4u * (uint32_t)r, yr[k]);
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    if (qwarp && gw != 0) named_bar_arrive(bid, 128);
-    else named_bar_sync(bid, 128);
-    if (i == 0) {   // A += (C G) C^T
+    if (issuer_warp) named_bar_sync(bar.bY, 128);
+    else named_bar_arrive(bar.bY, 128);
+    if (issuer) {   // X = Y G into T[:, P] (overwritten)
       tc_fence_after();
-      const uint64_t ch = desc_noswz(swb + SW_CH, 128, 256), cl = desc_noswz(swb + SW_CL, 128, 256);
-      const uint64_t qh = desc_noswz(swb + SW_CGH, 128, 256), ql = desc_noswz(swb + SW_CGL, 128, 256);
-      mma_bf16_ss(tA, qh, ch, kId128, 1u);
-      mma_bf16_ss(tA, qh, cl, kId128, 1u);
-      mma_bf16_ss(tA, ql, ch, kId128, 1u);
-      mma_commit(sbar);
+      const uint64_t a0 = desc_noswz(swb + SW_YH, 128, 256), a1 = desc_noswz(swb + SW_YM, 128, 256),
+                     a2 = desc_noswz(swb + SW_YL, 128, 256);
+      const uint64_t b0 = desc_noswz(swb + SW_GI, 128, 256), b1 = desc_noswz(swb + SW_GI + 512u, 128, 256),
+                     b2 = desc_noswz(swb + SW_GI + 1024u, 128, 256);
+      const uint32_t d = tA + p0;
+      mma_bf16_ss(d, a0, b0, kId16, 0u);
+      mma_bf16_ss(d, a0, b1, kId16, 1u);
+      mma_bf16_ss(d, a1, b0, kId16, 1u);
+      mma_bf16_ss(d, a0, b2, kId16, 1u);
+      mma_bf16_ss(d, a2, b0, kId16, 1u);
+      mma_bf16_ss(d, a1, b1, kId16, 1u);
+      mma_commit(bar.xbar);
     }
-    if (qwarp) {   // next block after this step, A_QQ + (C G)_Q C_Q^T, and its sweep
+    if (pwarp) {   // clear the P rows outside the P columns (those the X product writes)
+      const uint32_t sib = 16u * (uint32_t)(K ^ 1);   // P's sibling block in this warp's chunk of 32 columns
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        if (q == (K >> 1)) {
+          uint32_t v[16];
+          tmem_ld16(lb + tA + sib, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) v[t] = inP ? 0u : v[t];
+          tmem_st16(lb + tA + sib, v);
+        } else {
+          uint32_t v[32];
+          tmem_ld32(lb + tA + 32u * (uint32_t)q, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] = inP ? 0u : v[t];
+          tmem_st32(lb + tA + 32u * (uint32_t)q, v);
+        }
+      }
+    }
+    ok = mbar_wait(bar.xbar, xphase, abort_flag) && ok;
+    xphase ^= 1u;
+    tc_fence_after();
+    float x[16];
+    {
+      uint32_t v[16];
+      tmem_ld16(lb + tA + p0, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int t = 0; t < 16; ++t) x[t] = __uint_as_float(v[t]);
+      uint32_t z[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) z[t] = 0u;
+      tmem_st16(lb + tA + p0, z);   // T[:, P] = 0 before the update
+    }
+    store_row16_split3(swb + SW_XH, swb + SW_XM, swb + SW_XL, (uint32_t)i, x);
+    fence_proxy_async_smem();
+    tmem_wait_st();
+    tc_fence_before();
+    if (issuer_warp) named_bar_sync(bar.bX, 128);
+    else named_bar_arrive(bar.bX, 128);
+    if (issuer) {   // T += X Y^T, six products
+      tc_fence_after();
+      const uint64_t yh = desc_noswz(swb + SW_YH, 128, 256), ym = desc_noswz(swb + SW_YM, 128, 256),
+                     yl = desc_noswz(swb + SW_YL, 128, 256);
+      const uint64_t xh = desc_noswz(swb + SW_XH, 128, 256), xm = desc_noswz(swb + SW_XM, 128, 256),
+                     xl = desc_noswz(swb + SW_XL, 128, 256);
+      mma_bf16_ss(tA, xh, yh, kId128, 1u);
+      mma_bf16_ss(tA, xh, ym, kId128, 1u);
+      mma_bf16_ss(tA, xm, yh, kId128, 1u);
+      mma_bf16_ss(tA, xh, yl, kId128, 1u);
+      mma_bf16_ss(tA, xl, yh, kId128, 1u);
+      mma_bf16_ss(tA, xm, ym, kId128, 1u);
+      mma_commit(bar.sbar);
+    }
+    if (qwarp) {   // next block after this step, A_QQ + X_Q C_Q^T in fp32, and its sweep
       __syncwarp();
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
 #pragma unroll
         for (int t = 0; t < 16; t += 4) {
-          const float4 x = ld_shared_f4(cqb + 64u * (uint32_t)k + 4u * t);
-          aq[t] = fmaf(cg[k], x.x, aq[t]); aq[t + 1] = fmaf(cg[k], x.y, aq[t + 1]);
-          aq[t + 2] = fmaf(cg[k], x.z, aq[t + 2]); aq[t + 3] = fmaf(cg[k], x.w, aq[t + 3]);
+          const float4 cv = ld_shared_f4(cqb + 64u * (uint32_t)k + 4u * t);
+          aq[t] = fmaf(x[k], cv.x, aq[t]); aq[t + 1] = fmaf(x[k], cv.y, aq[t + 1]);
+          aq[t + 2] = fmaf(x[k], cv.z, aq[t + 2]); aq[t + 3] = fmaf(x[k], cv.w, aq[t + 3]);
         }
       }
       float gq[8];
       sweep16(aq, Kn & 1, lane, gq);
-      st_row8_f32(gnext + 64u * (uint32_t)r + 32u * (uint32_t)h, gq);
+      store_g_image(swb, r, h, gq);   // this step's X product has read the previous G
     }
-    bool ok = mbar_wait(sbar, sweep_phase, abort_flag);
-    sweep_phase ^= 1u;
-    tc_fence_after();
-    if (ok) {   // fix-ups of the pivot columns (all rows) and pivot rows
-      if (pwarp) {   // rewrite the full rows of this warp's 32 lanes
-        float gr[16];
-        if (inP) {
-#pragma unroll
-          for (int t = 0; t < 16; t += 4) {
-            const float4 x = ld_shared_f4(gcur + 64u * (uint32_t)r + 4u * t);
-            gr[t] = x.x; gr[t + 1] = x.y; gr[t + 2] = x.z; gr[t + 3] = x.w;
-          }
-        } else {
-#pragma unroll
-          for (int t = 0; t < 16; ++t) gr[t] = -cg[t];
-        }
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t v[32];
-          tmem_ld32(lb + tA + 32u * q, v);
-          tmem_wait_ld();
-          if (inP) {   // pivot rows: W_j^T for the columns outside P
-#pragma unroll
-            for (int t = 0; t < 32; t += 4) {
-              const float4 x = ld_shared_f4(swb + SW_W + (uint32_t)r * 512u + 4u * (uint32_t)(32 * q + t));
-              v[t] = __float_as_uint(x.x); v[t + 1] = __float_as_uint(x.y);
-              v[t + 2] = __float_as_uint(x.z); v[t + 3] = __float_as_uint(x.w);
-            }
-          }
-          if (q == (K >> 1)) {   // the 16 pivot columns sit in this 32-column chunk
-            if ((K & 1) == 0) {
-#pragma unroll
-              for (int t = 0; t < 16; ++t) v[t] = __float_as_uint(gr[t]);
-            } else {
-#pragma unroll
-              for (int t = 0; t < 16; ++t) v[16 + t] = __float_as_uint(gr[t]);
-            }
-          }
-          tmem_st32(lb + tA + 32u * q, v);
-        }
-      } else {
-        uint32_t v[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) v[t] = __float_as_uint(-cg[t]);
-        tmem_st16(lb + tA + p0, v);
-      }
-      tmem_wait_st();
-    }
-    tc_fence_before();
-    ok = named_bar_and(bend, 128, ok);
-    if (!ok) return false;
-    tc_fence_after();
   }
-  return true;
+  ok = mbar_wait(bar.sbar, sphase, abort_flag) && ok;   // the last step's update
+  sphase ^= 1u;
+  tc_fence_after();
+  return ok;
 }
 
 __global__ void __launch_bounds__(InvCfg::THREADS, 1)
@@ -566,14 +639,13 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::GROUPS * 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = warp >> 2, gw = warp & 3;
   const int i = gw * 32 + lane;
-  const uint32_t sbar = sbase + C::BAR_OFF + 8u * (uint32_t)g;
   if (tid == 0) {
-    for (int q = 0; q < C::GROUPS; ++q) mbar_init(sbase + C::BAR_OFF + 8u * q, 1);
+    for (int q = 0; q < C::NBAR; ++q) mbar_init(sbase + C::BAR_OFF + 8u * q, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -589,7 +661,9 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
   const uint32_t lb = (uint32_t)(gw * 32) << 16;
   const uint32_t swb = sbase + C::SW_BYTES * (uint32_t)g;
   const uint32_t bid = 1u + (uint32_t)g;
-  uint32_t sweep_phase = 0;
+  const InvBars bars{bid, 5u + (uint32_t)g, sbase + C::BAR_OFF + 8u * (uint32_t)g,
+                     sbase + C::BAR_OFF + 8u * (uint32_t)(C::GROUPS + g)};
+  uint32_t sphase = 0, xphase = 0;
 
   for (int m = blockIdx.x * C::GROUPS + g; m < FH; m += gridDim.x * C::GROUPS) {
     // row i of A -> TMEM lane i
@@ -615,7 +689,7 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
     tc_fence_before();
     named_bar_sync(bid, 128);
     tc_fence_after();
-    if (!sweep_inverse_tmem(tA, lb, swb, bid, bid + C::GROUPS, sbar, sweep_phase, abort_flag, i, gw, lane, g)) break;
+    const bool ok = sweep_inverse_tmem(tA, lb, swb, bars, sphase, xphase, abort_flag, i, gw, lane, g);
     // M = -(swept matrix): row i -> operand image row i (k index), debug copy
     uint8_t* img = Mimg + (size_t)m * kImgBytes;
 #pragma unroll 1
@@ -638,12 +712,13 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
     }
     // the next matrix overwrites these TMEM rows: every lane's reads first
     tc_fence_before();
-    named_bar_sync(bid, 128);
+    const bool all_ok = named_bar_and(bid, 128, ok);
     tc_fence_after();
+    if (!all_ok) break;
   }
-  if (i == 0) {   // the group's own tensor-core work completes before TMEM is released
-    mma_commit(sbar);
-    mbar_wait_drain(sbar, sweep_phase);
+  if (gw == g && lane == 0) {   // the group's own tensor-core work completes before TMEM is released
+    mma_commit(bars.sbar);
+    mbar_wait_drain(bars.sbar, sphase);
   }
   tc_fence_before();
   __syncthreads();
