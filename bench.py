@@ -382,7 +382,6 @@ def main():
 
     sampler = ClockSampler(local_rank)
     sampler.start()
-    timer = api.StageTimer(args.steps)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -395,8 +394,16 @@ def main():
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    stage_ms, calls = timer.read()
     ms = ev0.elapsed_time(ev1) / args.steps
+    # per-kernel device time: further steps of the same workload with CUDA
+    # events just before and after each launch, on its stream (kept out of the
+    # region above, so that the headline time carries no extra stream work)
+    kernel_steps = max(1, min(args.steps, 20))
+    timer = api.StageTimer(kernel_steps)
+    for _ in range(kernel_steps):
+        step()
+    torch.cuda.synchronize()
+    stage_ms, calls = timer.read()
     status = api.vda_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -493,6 +500,8 @@ def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches):
                                   else ""),
                    "per_rank_problem": "independent problem of the same size per GPU",
                    "l2": "inputs larger than L2 (about 3 GB read per step), no flush",
+                   "kernel_timing": f"events around each launch over {calls} further steps of this workload; "
+                                    "ms_per_step is timed without them",
                    "parallelism": f"replicas{world}"},
         "roofline": roofline,
         "op_roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof / (ms_max * 1e-3),

@@ -362,13 +362,14 @@ constexpr uint32_t SW_XH = 12288, SW_XM = 16384, SW_XL = 20480;   // X in three 
 constexpr uint32_t SW_GI = 24576;                                 // G in three parts, 3 x 512 B
 constexpr uint32_t SW_CQ = 26624;   // next block's rows of C, transposed, [2 steps][2 segments][16][16]
 
-// Pivot block swept at step s by group grp: the order 0,2,4,6,1,3,5,7 rotated
-// by grp.  The sweep's result does not depend on the order; this one puts
+// Pivot block swept at step s: the order 0,2,4,6,1,3,5,7 rotated by rot.  The
+// sweep's result does not depend on the order up to rounding; this one puts
 // consecutive blocks in different warps (a block's TMEM lanes belong to warp
-// block / 2, i.e. to a fixed sub-partition) and the groups' pivot warps of
-// one step on different sub-partitions.
-__device__ __forceinline__ int inv_block(int s, int grp) {
-  const int j = (s + grp) & 7;
+// block / 2, i.e. to a fixed sub-partition), and rotating it by the matrix
+// index spreads the pivot warps of the groups over the sub-partitions while
+// keeping each matrix's arithmetic independent of which group sweeps it.
+__device__ __forceinline__ int inv_block(int s, int rot) {
+  const int j = (s + rot) & 7;
   return j < 4 ? 2 * j : 2 * j - 7;
 }
 
@@ -465,12 +466,13 @@ struct InvBars {
 };
 
 // One warpgroup sweeps the matrix in TMEM columns [tA, tA + 128); thread i =
-// TMEM lane i; gw = warp index within the group, grp = group index.  Returns
-// false if a wait gave up (the matrix is then garbage; the barrier sequence is
-// still kept, so the group stays in step).
+// TMEM lane i; gw = warp index within the group, grp = group index, rot = the
+// rotation of the pivot order.  Returns false if a wait gave up (the matrix is
+// then garbage; the barrier sequence is still kept, so the group stays in
+// step).
 __device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t lb, uint32_t swb, const InvBars& bar,
                                                    uint32_t& sphase, uint32_t& xphase, volatile int* abort_flag,
-                                                   int i, int gw, int lane, int grp) {
+                                                   int i, int gw, int lane, int grp, int rot) {
   constexpr uint32_t kId128 = idesc_bf16(128, 128, 0, 0);
   constexpr uint32_t kId16 = idesc_bf16(128, 16, 0, 0);
   const int r = lane & 15, h = lane >> 4;
@@ -479,7 +481,7 @@ __device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t lb, uin
   bool ok = true;
   // G of the first pivot block (the matrix is untouched: P = its own block)
   {
-    const int K0 = inv_block(0, grp);
+    const int K0 = inv_block(0, rot);
     if (gw == (K0 >> 1)) {
       uint32_t v[16];
       tmem_ld16(lb + tA + 16u * (uint32_t)K0, v);
@@ -494,11 +496,11 @@ __device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t lb, uin
   }
 #pragma unroll 1
   for (int s = 0; s < 8; ++s) {
-    const int K = inv_block(s, grp);
+    const int K = inv_block(s, rot);
     const uint32_t p0 = 16u * (uint32_t)K;
     const bool inP = (i >> 4) == K;
     const bool pwarp = gw == (K >> 1);
-    const int Kn = inv_block(s + 1, grp);
+    const int Kn = inv_block(s + 1, rot);
     const bool qwarp = s < 7 && gw == (Kn >> 1);     // sweeps the next block ahead
     const bool inQ = qwarp && (i >> 4) == Kn;
     // by step parity: the sweeping warp of step s + 2 writes it only after
@@ -689,7 +691,7 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
     tc_fence_before();
     named_bar_sync(bid, 128);
     tc_fence_after();
-    const bool ok = sweep_inverse_tmem(tA, lb, swb, bars, sphase, xphase, abort_flag, i, gw, lane, g);
+    const bool ok = sweep_inverse_tmem(tA, lb, swb, bars, sphase, xphase, abort_flag, i, gw, lane, g, m & 3);
     // M = -(swept matrix): row i -> operand image row i (k index), debug copy
     uint8_t* img = Mimg + (size_t)m * kImgBytes;
 #pragma unroll 1
@@ -1491,10 +1493,14 @@ inline size_t tc_extra_workspace_bytes(bool tc, size_t FH, int d) {
 
 inline int tc_launches_per_forward() { return 4; }
 
-template <typename MarkFn>
+// The launch schedule on the caller's stream: Gram kernel, inverse, scan,
+// decay bridge (with a decay gate), readout.  Timer hooks begin(stage, stream)
+// / end(stage, stream) bracket each launch (stage 0 stats, 1 inverse, 2 scan,
+// 3 readout).
+template <typename Timer>
 int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_args& a, char* ws_AM,
               char* ws_B, char* ws_states, char* ws_img, char* ws_bridge, cudaStream_t s, float* stats_out,
-              MarkFn mark) {
+              Timer& timer) {
   const size_t FH = BH * (size_t)T;
   const size_t fdd = FH * tc::kDD;
   float* A = reinterpret_cast<float*>(ws_AM);
@@ -1502,19 +1508,22 @@ int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_
   float* st = reinterpret_cast<float*>(ws_states);
   uint8_t* img = reinterpret_cast<uint8_t*>(ws_img);
   int rc;
-  mark(0);
+  timer.begin(0, s);
   if ((rc = tc::launch_stats(a.k, a.v, a.beta, U, FH, A, Bt, s)) != VDA_OK) return rc;
+  timer.end(0, s);
   if ((rc = debug_check("stats", s)) != VDA_OK) return rc;
   if (stats_out &&
       (cudaMemcpyAsync(stats_out, A, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
        cudaMemcpyAsync(stats_out + fdd, Bt, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess))
     return VDA_ERR_CUDA;
-  mark(1);
+  timer.begin(1, s);
   if ((rc = tc::launch_inverse(A, FH, img, stats_out ? stats_out + 2 * fdd : nullptr, s)) != VDA_OK) return rc;
+  timer.end(1, s);
   if ((rc = debug_check("inverse", s)) != VDA_OK) return rc;
-  mark(2);
+  timer.begin(2, s);
   if ((rc = tc::launch_scan(img, Bt, a.S0_fwd, a.S0_rev, a.alpha, st, BH, T, chunk, NC, 2, s)) != VDA_OK)
     return rc;
+  timer.end(2, s);
   if ((rc = debug_check("scan", s)) != VDA_OK) return rc;
   float* bridge = nullptr;
   if (a.alpha) {   // products of the decay bridge (Eq. A.4), one per (b, h, frame, key channel)
@@ -1523,14 +1532,13 @@ int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_
     k_decay_bridge<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.alpha, (int)BH, T, tc::kD, chunk, window, bridge);
     if ((rc = launch_status("k_decay_bridge")) != VDA_OK) return rc;
   }
-  mark(3);
   const float eps = a.eps > 0.f ? a.eps : 1e-6f;
+  timer.begin(3, s);
   if ((rc = tc::launch_readout(a.q, a.gate, a.rms_weight, st, bridge, a.out, BH, T, U, chunk, NC, window, eps,
                                s)) != VDA_OK)
     return rc;
-  if ((rc = debug_check("readout", s)) != VDA_OK) return rc;
-  mark(4);
-  return VDA_OK;
+  timer.end(3, s);
+  return debug_check("readout", s);
 }
 
 // text state on the tensor-core kernels: stats over one frame of L tokens per

@@ -71,25 +71,39 @@ Plan make_plan(int B, int H, int T, int U, int d, int chunk, int window, int dty
 }
 
 // ----------------------------------------------------------------------------
-// per-stage timing (vda_timing_enable / vda_timing_read)
+// per-stage timing (vda_timing_enable / vda_timing_read): events just before
+// and just after each kernel launch, on the launch's stream
+constexpr int kMaxMarks = 16;   // timed launches per forward
 struct Timing {
   std::mutex mu;
   int max_calls = 0;
   int calls = 0;
-  std::vector<cudaEvent_t> ev;  // (kStages + 1) per call
-  std::vector<char> done;       // 1 once every event of the call's slot was recorded
+  std::vector<cudaEvent_t> ev;     // 2 * kMaxMarks per call: begin, end of each launch
+  std::vector<signed char> stage;  // kMaxMarks per call: the launch's stage, -1 when unused
+  std::vector<char> done;          // 1 once every event of the call's slot was recorded
 } g_timing;
-
-void timing_mark(int call_slot, int stage, cudaStream_t s) {
-  if (call_slot < 0) return;
-  cudaEventRecord(g_timing.ev[(size_t)call_slot * (kStages + 1) + stage], s);
-}
 
 int timing_begin_call() {
   std::lock_guard<std::mutex> lk(g_timing.mu);
   if (g_timing.max_calls <= 0 || g_timing.calls >= g_timing.max_calls) return -1;
   return g_timing.calls++;
 }
+
+// The timer one forward call hands to its launch schedule.
+struct CallTimer {
+  int slot = -1;
+  int n = 0;
+  void begin(int st, cudaStream_t s) {
+    if (slot < 0 || n >= kMaxMarks) return;
+    g_timing.stage[(size_t)slot * kMaxMarks + n] = (signed char)st;
+    cudaEventRecord(g_timing.ev[((size_t)slot * kMaxMarks + n) * 2], s);
+  }
+  void end(int, cudaStream_t s) {
+    if (slot < 0 || n >= kMaxMarks) return;
+    cudaEventRecord(g_timing.ev[((size_t)slot * kMaxMarks + n) * 2 + 1], s);
+    ++n;
+  }
+};
 
 // a forward that returns early leaves its slot incomplete: vda_timing_read skips it
 void timing_end_call(int call_slot) {
@@ -102,6 +116,7 @@ void timing_reset_locked() {
   for (cudaEvent_t e : g_timing.ev)
     if (e) cudaEventDestroy(e);
   g_timing.ev.clear();
+  g_timing.stage.clear();
   g_timing.done.clear();
   g_timing.calls = 0;
   g_timing.max_calls = 0;
@@ -109,7 +124,7 @@ void timing_reset_locked() {
 
 // ----------------------------------------------------------------------------
 template <int D, typename TIo>
-int launch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, int tslot,
+int launch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, CallTimer& tm,
                 float* stats_out) {
   float* AM = reinterpret_cast<float*>(ws + p.off_AM);
   float* Bm = reinterpret_cast<float*>(ws + p.off_B);
@@ -117,29 +132,31 @@ int launch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, int 
   const size_t fdd = p.FH * (size_t)D * D;
   float* bridge = a.alpha ? reinterpret_cast<float*>(ws + p.off_bridge) : nullptr;
 
-  timing_mark(tslot, 0, s);
+  tm.begin(0, s);
   vda::k_stats_simt<D, TIo><<<(unsigned)p.FH, 256, 0, s>>>(
       static_cast<const TIo*>(a.k), static_cast<const TIo*>(a.v), a.beta, p.U, AM, Bm);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  tm.end(0, s);
   if (stats_out) {
     if (cudaMemcpyAsync(stats_out, AM, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(stats_out + fdd, Bm, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
       return VDA_ERR_CUDA;
   }
-  timing_mark(tslot, 1, s);
+  tm.begin(1, s);
   vda::k_gj_inverse<D><<<(unsigned)p.FH, 256, 0, s>>>(AM);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  tm.end(1, s);
   if (stats_out) {
     if (cudaMemcpyAsync(stats_out + 2 * fdd, AM, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
       return VDA_ERR_CUDA;
   }
-  timing_mark(tslot, 2, s);
+  tm.begin(2, s);
   constexpr int RB = 16;
   dim3 gs((unsigned)p.BH, 2, D / RB);
   vda::k_scan_simt<D, RB><<<gs, D, 0, s>>>(AM, Bm, a.S0_fwd, a.S0_rev, a.alpha, st, (int)p.BH, p.T,
                                            p.chunk, p.NC);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
-  timing_mark(tslot, 3, s);
+  tm.end(2, s);
   if (bridge) {
     const size_t n = p.FH * (size_t)D;
     vda::k_decay_bridge<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.alpha, (int)p.BH, p.T, D, p.chunk, p.window,
@@ -162,21 +179,22 @@ int launch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, int 
   splits = std::max(1, std::min(splits, 65535));
   dim3 gr((unsigned)pairs, (unsigned)splits);
   const float eps = a.eps > 0.f ? a.eps : 1e-6f;
+  tm.begin(3, s);
   vda::k_readout_simt<D, TIo><<<gr, 256, smem, s>>>(
       static_cast<const TIo*>(a.q), static_cast<const TIo*>(a.gate), a.rms_weight, st, bridge,
       static_cast<TIo*>(a.out), (int)p.BH, p.T, p.U, p.chunk, p.NC, p.window, eps);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
-  timing_mark(tslot, 4, s);
+  tm.end(3, s);
   return VDA_OK;
 }
 
 template <typename TIo>
-int dispatch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, int tslot, float* so) {
+int dispatch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, CallTimer& tm, float* so) {
   switch (p.d) {
-    case 16: return launch_simt<16, TIo>(p, a, ws, s, tslot, so);
-    case 32: return launch_simt<32, TIo>(p, a, ws, s, tslot, so);
-    case 64: return launch_simt<64, TIo>(p, a, ws, s, tslot, so);
-    case 128: return launch_simt<128, TIo>(p, a, ws, s, tslot, so);
+    case 16: return launch_simt<16, TIo>(p, a, ws, s, tm, so);
+    case 32: return launch_simt<32, TIo>(p, a, ws, s, tm, so);
+    case 64: return launch_simt<64, TIo>(p, a, ws, s, tm, so);
+    case 128: return launch_simt<128, TIo>(p, a, ws, s, tm, so);
   }
   return VDA_ERR_UNSUPPORTED;
 }
@@ -196,20 +214,20 @@ int validate_args(const vda_args* a) {
 
 int forward_impl(const vda_args& a, char* ws, const Plan& p, float* states_out, float* stats_out) {
   cudaStream_t s = static_cast<cudaStream_t>(a.stream);
-  const int tslot = timing_begin_call();
+  CallTimer tm;
+  tm.slot = timing_begin_call();
   int rc;
   if (p.tc) {
     rc = vda::launch_tc(p.BH, p.T, p.U, p.chunk, p.NC, p.window, a, ws + p.off_AM, ws + p.off_B,
                         ws + p.off_states, ws + p.total - vda::tc_extra_workspace_bytes(true, p.FH, p.d),
-                        ws + p.off_bridge, s, stats_out,
-                        [&](int stage) { timing_mark(tslot, stage, s); });
+                        ws + p.off_bridge, s, stats_out, tm);
   } else if (p.dtype == VDA_BF16) {
-    rc = dispatch_simt<__nv_bfloat16>(p, a, ws, s, tslot, stats_out);
+    rc = dispatch_simt<__nv_bfloat16>(p, a, ws, s, tm, stats_out);
   } else {
-    rc = dispatch_simt<float>(p, a, ws, s, tslot, stats_out);
+    rc = dispatch_simt<float>(p, a, ws, s, tm, stats_out);
   }
   if (rc != VDA_OK) return rc;
-  timing_end_call(tslot);
+  timing_end_call(tm.slot);
   if (states_out) {
     const size_t bytes = 2 * p.BH * (size_t)(p.NC + 1) * p.d * p.d * sizeof(float);
     if (cudaMemcpyAsync(states_out, ws + p.off_states, bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
@@ -627,7 +645,8 @@ int vda_timing_enable(int max_calls) {
   std::lock_guard<std::mutex> lk(g_timing.mu);
   timing_reset_locked();
   if (max_calls <= 0) return VDA_OK;
-  g_timing.ev.assign((size_t)max_calls * (kStages + 1), nullptr);
+  g_timing.ev.assign((size_t)max_calls * kMaxMarks * 2, nullptr);
+  g_timing.stage.assign((size_t)max_calls * kMaxMarks, (signed char)-1);
   g_timing.done.assign((size_t)max_calls, 0);
   for (auto& e : g_timing.ev)
     if (cudaEventCreate(&e) != cudaSuccess) {
@@ -645,12 +664,16 @@ int vda_timing_read(float* stage_ms, int n_stages, int* calls) {
   int rc = VDA_OK, complete = 0;
   for (int c = 0; c < g_timing.calls && rc == VDA_OK; ++c) {
     if (!g_timing.done[(size_t)c]) continue;   // a forward that failed part-way
-    cudaEvent_t* e = &g_timing.ev[(size_t)c * (kStages + 1)];
-    if (cudaEventSynchronize(e[kStages]) != cudaSuccess) { rc = VDA_ERR_CUDA; break; }
-    for (int st = 0; st < std::min(n_stages, kStages); ++st) {
+    for (int n = 0; n < kMaxMarks && rc == VDA_OK; ++n) {
+      const int st = g_timing.stage[(size_t)c * kMaxMarks + n];
+      if (st < 0) break;
+      cudaEvent_t* e = &g_timing.ev[((size_t)c * kMaxMarks + n) * 2];
       float ms = 0.f;
-      if (cudaEventElapsedTime(&ms, e[st], e[st + 1]) != cudaSuccess) { rc = VDA_ERR_CUDA; break; }
-      stage_ms[st] += ms;
+      if (cudaEventSynchronize(e[1]) != cudaSuccess || cudaEventElapsedTime(&ms, e[0], e[1]) != cudaSuccess) {
+        rc = VDA_ERR_CUDA;
+        break;
+      }
+      if (st < n_stages) stage_ms[st] += ms;
     }
     ++complete;
   }

@@ -201,10 +201,11 @@ VDA_API int vda_device_status(void* stream);
 VDA_API int vda_selftest_wait_timeout(int max_polls, void* stream);
 
 /* Per-stage device timing for profiling.  vda_timing_enable(n) makes the next
- * n forward calls record CUDA events between their stages (stats, inverse,
- * scan, readout) on the call's stream; vda_timing_read(ms, 4, &calls)
- * synchronises on the recorded events and writes the summed milliseconds of
- * each stage and the number of calls recorded, then disables timing.
+ * n forward calls record a CUDA event just before and just after each kernel
+ * launch, on the launch's stream; vda_timing_read(ms, 4, &calls) synchronises
+ * on the recorded events and writes, per stage (stats, inverse, scan,
+ * readout), the milliseconds summed over that stage's launches and calls, and
+ * the number of calls recorded, then disables timing and releases the events.
  * vda_timing_enable(0) disables it. */
 VDA_API int vda_timing_enable(int max_calls);
 VDA_API int vda_timing_read(float* stage_ms, int n_stages, int* calls);
