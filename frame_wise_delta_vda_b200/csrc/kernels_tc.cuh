@@ -17,6 +17,7 @@
 
 #include <cstdio>
 #include <cstdlib>
+#include <utility>
 
 #include "common.cuh"
 #include "kernels_simt.cuh"
@@ -157,6 +158,12 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // launched after the previous grid with programmatic serialisation: the
+  // prologue above overlapped its tail; its results are visible from here.
+  // Only then may the next grid start, so that every CTA of this one is
+  // resident before a CTA of the next can take an SM
+  grid_wait_prerequisites();
+  grid_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const int nt = (U + C::UT - 1) / C::UT;
   int last_it[C::NST];   // producer: last iteration issued on each stage
@@ -658,6 +665,8 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_wait_prerequisites();   // the Gram kernel's A is complete (see k_stats_tc)
+  grid_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tA = tmem + C::TCOLS * (uint32_t)g;
   const uint32_t lb = (uint32_t)(gw * 32) << 16;
@@ -817,6 +826,8 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  grid_wait_prerequisites();   // M images and B are complete (see k_stats_tc)
+  grid_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   auto frame_of = [&](int i) { return dir == 0 ? i : T - 1 - i; };
   int last_i[2] = {-1, -1};   // producer: last step issued on each stage
@@ -1061,12 +1072,15 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (tid < kD) sw[tid] = 0.5f * w[tid];
   if (warp == C::WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), 256);
     tmem_relinquish();
   }
   tc_fence_before();
+  __syncthreads();
+  grid_wait_prerequisites();   // boundary states are complete (see k_stats_tc)
+  grid_launch_dependents();
+  if (tid < kD) sw[tid] = 0.5f * w[tid];
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -1402,6 +1416,31 @@ inline bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch with programmatic stream serialisation: the kernel's CTAs may start
+// while the previous grid on the stream finishes; each of the four kernels
+// waits for that grid (griddepcontrol.wait) before reading what it wrote.
+template <typename... Params, typename... Args>
+inline int launch_pdl(const char* name, void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) {
+    cudaGetLastError();   // reported through the status instead
+    if (debug_sync_enabled()) fprintf(stderr, "vda: launch of %s failed: %s\n", name, cudaGetErrorString(e));
+    return VDA_ERR_CUDA;
+  }
+  return launch_status(name);
+}
+
 inline int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -1420,8 +1459,8 @@ inline int launch_stats(const void* K, const void* V, const float* beta, int U, 
       cudaSuccess)
     return launch_status("k_stats_tc (shared-memory attribute)");
   const int grid = (int)std::min<size_t>(FH, (size_t)num_sms());
-  k_stats_tc<<<grid, StatsCfg::THREADS, StatsCfg::SMEM, s>>>(tmK, tmV, beta, U, (int)FH, A, B);
-  return launch_status("k_stats_tc");
+  return launch_pdl("k_stats_tc", k_stats_tc, dim3(grid), dim3(StatsCfg::THREADS), StatsCfg::SMEM, s, tmK, tmV, beta,
+                    U, (int)FH, A, B);
 }
 
 // M = (I + A)^{-1} images (and optional fp32 copy) for FH matrices
@@ -1431,8 +1470,8 @@ inline int launch_inverse(const float* A, size_t FH, uint8_t* Mimg, float* M_dbg
     return launch_status("k_inverse_tc (shared-memory attribute)");
   const size_t per_cta = (size_t)InvCfg::GROUPS;
   const int grid = (int)std::min<size_t>((FH + per_cta - 1) / per_cta, (size_t)num_sms());
-  k_inverse_tc<<<grid, InvCfg::THREADS, InvCfg::SMEM, s>>>(A, (int)FH, Mimg, M_dbg);
-  return launch_status("k_inverse_tc");
+  return launch_pdl("k_inverse_tc", k_inverse_tc, dim3(grid), dim3(InvCfg::THREADS), InvCfg::SMEM, s, A, (int)FH,
+                    Mimg, M_dbg);
 }
 
 inline int launch_scan(const uint8_t* Mimg, const float* Bm, const float* S0f, const float* S0r,
@@ -1442,9 +1481,8 @@ inline int launch_scan(const uint8_t* Mimg, const float* Bm, const float* S0f, c
       cudaSuccess)
     return VDA_ERR_CUDA;
   dim3 grid((unsigned)BH, (unsigned)ndir);
-  k_scan_tc<<<grid, ScanCfg::THREADS, ScanCfg::SMEM, s>>>(Mimg, Bm, S0f, S0r, alpha, states, (int)BH, T, chunk,
-                                                          NC);
-  return launch_status("k_scan_tc");
+  return launch_pdl("k_scan_tc", k_scan_tc, grid, dim3(ScanCfg::THREADS), ScanCfg::SMEM, s, Mimg, Bm, S0f, S0r,
+                    alpha, states, (int)BH, T, chunk, NC);
 }
 
 inline int launch_readout(const void* Q, const void* G, const float* w, const float* states, const float* bridge,
@@ -1473,9 +1511,8 @@ inline int launch_readout(const void* Q, const void* G, const float* w, const fl
       cudaSuccess)
     return VDA_ERR_CUDA;
   const int grid = (int)std::min<long long>(g.total, (long long)num_sms());
-  k_readout_tc<<<grid, ReadoutCfg::THREADS, ReadoutCfg::SMEM, s>>>(
-      tmQ, tmG, tmO, w, states, bridge, static_cast<__nv_bfloat16*>(out), g, eps);
-  return launch_status("k_readout_tc");
+  return launch_pdl("k_readout_tc", k_readout_tc, dim3(grid), dim3(ReadoutCfg::THREADS), ReadoutCfg::SMEM, s, tmQ,
+                    tmG, tmO, w, states, bridge, static_cast<__nv_bfloat16*>(out), g, eps);
 }
 
 }  // namespace tc
