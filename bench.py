@@ -56,6 +56,11 @@ def parse():
                     help="workload to run (the benchmark line is defined on 'full'; other "
                          "workloads serve profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layout", choices=["replicas", "heads"], default="replicas",
+                    help="replicas: every rank runs its own problem of the full size (weak scaling, no "
+                         "collective); heads: one problem, each rank holding a token shard for every head, "
+                         "exchanged into head shards and back by all-to-all around the forward (strong "
+                         "scaling; H and T*U divisible by the rank count)")
     ap.add_argument("--prep", action="store_true",
                     help="time the feature preparation (vda_prep) on the full-size shapes instead of the forward")
     return ap.parse_args()
@@ -351,8 +356,10 @@ def main():
     if args.workload not in gen.WORKLOADS:
         raise SystemExit(f"{args.workload} is a feature-preparation workload: use --prep")
     base = gen.WORKLOADS[args.workload]
-    # every rank runs its own problem of the same size (weak scaling)
-    wl = gen.Workload(**{**base.__dict__, "seed": ranks.rank_seed(base.seed, rank)})
+    heads = args.layout == "heads"
+    # replicas: every rank runs its own problem of the same size (weak
+    # scaling); heads: every rank holds a token shard of the one problem
+    wl = base if heads else gen.Workload(**{**base.__dict__, "seed": ranks.rank_seed(base.seed, rank)})
 
     x = gen.make_inputs(wl)
     if "k_text" not in x:
@@ -363,17 +370,42 @@ def main():
             return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
         return torch.from_numpy(a).to(dev)
 
-    t = {k: dev_t(v) for k, v in x.items() if v is not None}
-    S0 = api.vda_text_state(t["k_text"], t["v_text"], t["beta_text"]) if "k_text" in t else None
-    out = torch.empty_like(t["q"])
-    ws = api.workspace_for(t["q"], t["v"], wl.chunk)
     stream = torch.cuda.current_stream()
+    if not heads:
+        t = {k: dev_t(v) for k, v in x.items() if v is not None}
+        S0 = api.vda_text_state(t["k_text"], t["v_text"], t["beta_text"]) if "k_text" in t else None
+        out = torch.empty_like(t["q"])
+        ws = api.workspace_for(t["q"], t["v"], wl.chunk)
+        alpha = t.get("alpha")
+        wl_rank = wl
 
-    alpha = t.get("alpha")
+        def step():
+            api.vda_forward(t["q"], t["k"], t["v"], t["beta"], t["gate"], t["rms_weight"], S0, S0,
+                            chunk=wl.chunk, window_chunks=wl.window_chunks, out=out, workspace=ws, alpha=alpha)
+    else:
+        from frame_wise_delta_vda_b200 import ulysses
+        if wl.H % world or (wl.T * wl.U) % world:
+            raise SystemExit(f"--layout heads needs H = {wl.H} and T*U = {wl.T * wl.U} divisible by {world}")
+        Hp = wl.H // world
+        hs = slice(rank * Hp, (rank + 1) * Hp)
+        host = {k: torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v)
+                for k, v in x.items() if v is not None}
+        for k in ("q", "k", "v", "gate", "k_text", "v_text"):
+            if k in host:
+                host[k] = host[k].view(torch.bfloat16)
+        t = {k: ulysses.token_shard(host[k], rank, world, wl.T, wl.U).to(dev) for k in ("q", "k", "v", "gate", "beta")}
+        t["rms_weight"] = host["rms_weight"].to(dev)
+        S0 = (api.vda_text_state(host["k_text"][:, hs].contiguous().to(dev), host["v_text"][:, hs].contiguous().to(dev),
+                                 host["beta_text"][:, hs].contiguous().to(dev)) if "k_text" in host else None)
+        alpha = host["alpha"][:, hs].contiguous().to(dev) if "alpha" in host else None
+        out = torch.empty((wl.B, Hp, wl.T, wl.U, wl.d), dtype=torch.bfloat16, device=dev)
+        ws = api.workspace_for(out, out, wl.chunk)
+        wl_rank = gen.Workload(**{**wl.__dict__, "H": Hp})
+        del host
 
-    def step():
-        api.vda_forward(t["q"], t["k"], t["v"], t["beta"], t["gate"], t["rms_weight"], S0, S0,
-                        chunk=wl.chunk, window_chunks=wl.window_chunks, out=out, workspace=ws, alpha=alpha)
+        def step():
+            ulysses.vda_forward_ulysses(t["q"], t["k"], t["v"], t["beta"], t["gate"], t["rms_weight"], S0, S0,
+                                        wl.T, wl.U, wl.chunk, wl.window_chunks, alpha=alpha, out=out, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -410,13 +442,13 @@ def main():
 
     ms_max = ranks.max_over_ranks(ms, dist if world > 1 else None, dev)
     # a decay gate adds one launch per forward (the bridge products)
-    launches = (api.vda_launches_per_forward(wl.B, wl.H, wl.T, wl.U, wl.d, wl.d, wl.chunk)
+    launches = (api.vda_launches_per_forward(wl_rank.B, wl_rank.H, wl.T, wl.U, wl.d, wl.d, wl.chunk)
                 + (1 if alpha is not None else 0)) * args.steps
 
     # ---- end to end through the host-buffer entry point ------------------------
     e2e_steps = args.e2e_steps if args.e2e_steps is not None else max(3, min(args.steps, 10))
     e2e = None
-    if e2e_steps > 0:
+    if e2e_steps > 0 and not heads:
         e2e = run_e2e(api, x, S0, out, wl, dev, e2e_steps, world, dist)
 
     if world > 1:
@@ -424,7 +456,7 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
-    emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches)
+    emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches, wl_rank=wl_rank)
 
 
 def run_e2e(api, x, S0, out, wl, dev, e2e_steps, world, dist):
@@ -461,11 +493,16 @@ def run_e2e(api, x, S0, out, wl, dev, e2e_steps, world, dist):
     return {"e2e_s": e2e_s, "h2d": h2d, "d2h": d2h}
 
 
-def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches):
+def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches, wl_rank=None):
+    """The JSON line.  wl: the workload of the metric (each rank's own problem
+    with replicas, the one sharded problem with heads); wl_rank: the problem
+    one rank's kernels process (for the roofline)."""
+    heads = getattr(args, "layout", "replicas") == "heads"
+    wl_rank = wl_rank or wl
 
     # ---- roofline of the dominant kernel ------------------------------------
     peaks, peak_src = load_peaks()
-    alg = algorithmic(wl)
+    alg = algorithmic(wl_rank)
     dom = max(stage_ms, key=stage_ms.get)
     dom_ms = stage_ms[dom] / max(calls, 1)
     limiter, kname, _ = stage_kernels(wl)[dom]
@@ -486,23 +523,24 @@ def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches):
     t_roof = max(alg["op"]["bytes"] / (peaks["hbm_gbs"] * 1e9),
                  alg["op"]["flops"] / (peaks["bf16_tflops"] * 1e12))
 
-    tokens = wl.tokens * world
+    tokens = wl.tokens if heads else wl.tokens * world
     line = {
         "metric": METRIC, "value": tokens / (ms_max * 1e-3), "unit": UNIT, "n_gpus": world,
         "head_tokens_per_s": tokens * wl.H / (ms_max * 1e-3),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong" if heads else "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"{wl.name}: B={wl.B} H={wl.H} T={wl.T} U={wl.U} d={wl.d} chunk={wl.chunk} "
                                f"window=+-{wl.window_chunks}"
                                + (f", text S0 from {wl.text_tokens} prompt tokens" if wl.text_tokens else ", S0 = 0")
                                + (f", decay gate alpha = sigmoid(N({wl.alpha_mean}, 1))" if wl.alpha_mean is not None
                                   else ""),
-                   "per_rank_problem": "independent problem of the same size per GPU",
+                   "per_rank_problem": (f"token shard of one problem, {wl_rank.H} heads per GPU after the "
+                                        "all-to-all" if heads else "independent problem of the same size per GPU"),
                    "l2": "inputs larger than L2 (about 3 GB read per step), no flush",
                    "kernel_timing": f"events around each launch over {calls} further steps of this workload; "
                                     "ms_per_step is timed without them",
-                   "parallelism": f"replicas{world}"},
+                   "parallelism": f"heads{world} (all-to-all)" if heads else f"replicas{world}"},
         "roofline": roofline,
         "op_roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof / (ms_max * 1e-3),
                         "bytes": alg["op"]["bytes"], "flops": alg["op"]["flops"]},

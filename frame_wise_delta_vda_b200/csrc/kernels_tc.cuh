@@ -1458,7 +1458,12 @@ inline int launch_stats(const void* K, const void* V, const float* beta, int U, 
   if (cudaFuncSetAttribute(k_stats_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StatsCfg::SMEM) !=
       cudaSuccess)
     return launch_status("k_stats_tc (shared-memory attribute)");
-  const int grid = (int)std::min<size_t>(FH, (size_t)num_sms());
+  // as many rounds as num_sms CTAs need, over as few CTAs as keep that count:
+  // every CTA then takes the same number of frame-heads (2880 = 144 x 20 at
+  // full size) instead of a last, partial round on part of the SMs
+  const size_t sms = (size_t)num_sms();
+  const size_t rounds = (FH + sms - 1) / sms;
+  const int grid = (int)((FH + rounds - 1) / rounds);
   return launch_pdl("k_stats_tc", k_stats_tc, dim3(grid), dim3(StatsCfg::THREADS), StatsCfg::SMEM, s, tmK, tmV, beta,
                     U, (int)FH, A, B);
 }
