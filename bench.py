@@ -61,6 +61,12 @@ def parse():
                          "collective); heads: one problem, each rank holding a token shard for every head, "
                          "exchanged into head shards and back by all-to-all around the forward (strong "
                          "scaling; H and T*U divisible by the rank count)")
+    ap.add_argument("--scan-form", choices=["auto", "frames", "chunks"], default="auto",
+                    help="scan form of the tensor-core path: per-frame chains, chunk-wise (compose the "
+                         "chunks' maps, then scan them), or the library's choice")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the workload with this many heads instead of its own (e.g. 6: the per-GPU "
+                         "load of an 8-way head split of 48 heads)")
     ap.add_argument("--prep", action="store_true",
                     help="time the feature preparation (vda_prep) on the full-size shapes instead of the forward")
     return ap.parse_args()
@@ -356,6 +362,8 @@ def main():
     if args.workload not in gen.WORKLOADS:
         raise SystemExit(f"{args.workload} is a feature-preparation workload: use --prep")
     base = gen.WORKLOADS[args.workload]
+    if args.heads is not None:
+        base = gen.Workload(**{**base.__dict__, "H": args.heads, "name": f"{base.name}_H{args.heads}"})
     heads = args.layout == "heads"
     # replicas: every rank runs its own problem of the same size (weak
     # scaling); heads: every rank holds a token shard of the one problem
@@ -381,7 +389,8 @@ def main():
 
         def step():
             api.vda_forward(t["q"], t["k"], t["v"], t["beta"], t["gate"], t["rms_weight"], S0, S0,
-                            chunk=wl.chunk, window_chunks=wl.window_chunks, out=out, workspace=ws, alpha=alpha)
+                            chunk=wl.chunk, window_chunks=wl.window_chunks, out=out, workspace=ws, alpha=alpha,
+                            scan_form=args.scan_form)
     else:
         from frame_wise_delta_vda_b200 import ulysses
         if wl.H % world or (wl.T * wl.U) % world:
@@ -405,7 +414,8 @@ def main():
 
         def step():
             ulysses.vda_forward_ulysses(t["q"], t["k"], t["v"], t["beta"], t["gate"], t["rms_weight"], S0, S0,
-                                        wl.T, wl.U, wl.chunk, wl.window_chunks, alpha=alpha, out=out, workspace=ws)
+                                        wl.T, wl.U, wl.chunk, wl.window_chunks, alpha=alpha, out=out, workspace=ws,
+                                        scan_form=args.scan_form)
 
     for _ in range(args.warmup):
         step()
@@ -442,8 +452,11 @@ def main():
 
     ms_max = ranks.max_over_ranks(ms, dist if world > 1 else None, dev)
     # a decay gate adds one launch per forward (the bridge products)
-    launches = (api.vda_launches_per_forward(wl_rank.B, wl_rank.H, wl.T, wl.U, wl.d, wl.d, wl.chunk)
-                + (1 if alpha is not None else 0)) * args.steps
+    # (the chunk-wise scans take two launches)
+    per_fwd = api.vda_launches_per_forward(wl_rank.B, wl_rank.H, wl.T, wl.U, wl.d, wl.d, wl.chunk)
+    if args.scan_form != "auto" and wl.d == 128 and wl.dtype == "bf16":
+        per_fwd = 5 if args.scan_form == "chunks" else 4
+    launches = (per_fwd + (1 if alpha is not None else 0)) * args.steps
 
     # ---- end to end through the host-buffer entry point ------------------------
     e2e_steps = args.e2e_steps if args.e2e_steps is not None else max(3, min(args.steps, 10))
@@ -540,7 +553,8 @@ def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches, wl_ran
                    "l2": "inputs larger than L2 (about 3 GB read per step), no flush",
                    "kernel_timing": f"events around each launch over {calls} further steps of this workload; "
                                     "ms_per_step is timed without them",
-                   "parallelism": f"heads{world} (all-to-all)" if heads else f"replicas{world}"},
+                   "parallelism": f"heads{world} (all-to-all)" if heads else f"replicas{world}",
+                   "scan_form": getattr(args, "scan_form", "auto")},
         "roofline": roofline,
         "op_roofline": {"t_roof_us": t_roof * 1e6, "frac": t_roof / (ms_max * 1e-3),
                         "bytes": alg["op"]["bytes"], "flops": alg["op"]["flops"]},

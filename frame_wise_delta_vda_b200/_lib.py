@@ -22,6 +22,9 @@ VDA_ERR_CUDA = 4
 VDA_ERR_TIMEOUT = 5
 VDA_BF16 = 0
 VDA_F32 = 1
+VDA_SCAN_AUTO = 0
+VDA_SCAN_FRAMES = 1
+VDA_SCAN_CHUNKS = 2
 NOALLOC_SCRATCH_BYTES = 16 << 20   # VDA_NOALLOC_SCRATCH_BYTES in include/vda.h
 
 c_int, c_size_t, c_void_p, c_float = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
@@ -40,6 +43,7 @@ class VdaArgs(ctypes.Structure):
         ("eps", c_float),
         ("stream", c_void_p),
         ("alpha", c_void_p),
+        ("scan_form", c_int),
     ]
 
 

@@ -11,7 +11,10 @@ import ctypes
 
 import torch
 
-from ._lib import VDA_BF16, VDA_F32, VdaArgs, VdaError, VdaPrepArgs, check, lib  # noqa: F401
+from ._lib import (VDA_BF16, VDA_F32, VDA_SCAN_AUTO, VDA_SCAN_CHUNKS, VDA_SCAN_FRAMES, VdaArgs,  # noqa: F401
+                   VdaError, VdaPrepArgs, check, lib)
+
+_SCAN_FORMS = {"auto": VDA_SCAN_AUTO, "frames": VDA_SCAN_FRAMES, "chunks": VDA_SCAN_CHUNKS}
 
 _DTYPES = {torch.bfloat16: VDA_BF16, torch.float32: VDA_F32}
 
@@ -47,7 +50,7 @@ def _check_tensor(name, t, dtype=None, shape=None, device=None, allow_none=False
 
 
 def make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks,
-              eps=1e-6, stream=None, check_device=True, alpha=None):
+              eps=1e-6, stream=None, check_device=True, alpha=None, scan_form="auto"):
     """Build the C `vda_args` block from tensors (device or host)."""
     if q.dim() != 5:
         raise ValueError("q must be [B, H, T, U, d_k]")
@@ -81,6 +84,9 @@ def make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, windo
     a.eps = float(eps)
     a.stream = _stream(stream).value if check_device else None
     a.alpha = alpha.data_ptr() if alpha is not None else None
+    if scan_form not in _SCAN_FORMS:
+        raise ValueError(f"scan_form must be one of {sorted(_SCAN_FORMS)}")
+    a.scan_form = _SCAN_FORMS[scan_form]
     return a
 
 
@@ -97,19 +103,22 @@ def workspace_for(q, v, chunk):
 
 def vda_forward(q, k, v, beta, gate, rms_weight, S0_fwd=None, S0_rev=None, chunk=5,
                 window_chunks=1, out=None, workspace=None, states_out=None, stats_out=None,
-                eps=1e-6, stream=None, alpha=None):
+                eps=1e-6, stream=None, alpha=None, scan_form="auto"):
     """Bidirectional VDA forward (see include/vda.h).  Returns `out`.
 
-    Without `workspace`, `states_out`, `stats_out` or `alpha` this calls
-    `vda_forward` / `vda_forward_f32` (stream-ordered workspace); otherwise
-    `vda_forward_ex`.  `alpha` [B, H, T, d_k] float32 adds the decay gate.
+    Without `workspace`, `states_out`, `stats_out`, `alpha` or a `scan_form`
+    other than "auto" this calls `vda_forward` / `vda_forward_f32`
+    (stream-ordered workspace); otherwise `vda_forward_ex`.  `alpha`
+    [B, H, T, d_k] float32 adds the decay gate; `scan_form` ("auto", "frames",
+    "chunks") selects the scan form of the tensor-core path.
     """
     if out is None:
         out = torch.empty(q.shape[:-1] + (v.shape[-1],), dtype=q.dtype, device=q.device)
     a = make_args(q, k, v, beta, gate, rms_weight, S0_fwd, S0_rev, out, chunk, window_chunks, eps, stream,
-                  alpha=alpha)
+                  alpha=alpha, scan_form=scan_form)
     L = lib()
-    if workspace is None and states_out is None and stats_out is None and eps == 1e-6 and alpha is None:
+    if (workspace is None and states_out is None and stats_out is None and eps == 1e-6 and alpha is None
+            and scan_form == "auto"):
         fn = L.vda_forward if a.dtype == VDA_BF16 else L.vda_forward_f32
         rc = fn(a.q, a.k, a.v, a.beta, a.gate, a.rms_weight, a.S0_fwd, a.S0_rev,
                 a.B, a.H, a.T, a.U, a.d_k, a.d_v, a.chunk, a.window_chunks, a.out, a.stream)

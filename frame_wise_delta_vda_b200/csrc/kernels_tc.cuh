@@ -760,7 +760,35 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
 // Warp 8: bulk-copies the M image of the coming steps (two stages).
 // Warp 9: MMA issuer, TMEM owner.
 // Boundary states: fwd[j] after frames [0, jC), rev[j] after [jC, T).
+//
+// The same kernel body runs the chunk-wise form of the scans (Section 5,
+// "Chunk-wise scans"; Appendix A.1): frame t acts on a state as the affine map
+// S -> S (Diag(alpha_t) M_t) + B_t M_t, so the frames of chunk c compose, in
+// the direction's order, into S -> S P_c + J_c.
+//   kScanCompose: one CTA per (b, h, chunk, direction, part) runs the chunk's
+//     frames from S = 0 with the B_t (part J: gives J_c) or from S = I
+//     without them (part P: gives P_c).  The four CTAs of a chunk are
+//     neighbours and share its M images and B through L2.  J_c is stored in
+//     fp32, P_c as the M operand image (bf16 hi / lo).
+//   kScanChunks: one CTA per chain runs the NC chunk maps,
+//     S <- S P_c + J_c, and stores every boundary state.
+// The sequential chain shrinks from T steps to C + NC steps at about twice
+// the tensor-core work (the P_c products), which pays when few chains run.
 // ===========================================================================
+enum ScanMode { kScanFrames = 0, kScanCompose = 1, kScanChunks = 2 };
+
+struct ScanArgs {
+  const uint8_t* Mimg;   // frames, compose: M images [BH][T]; chunks: P_c images [2][BH][NC]
+  const float* Bm;       // frames, compose: B_t [BH][T]; chunks: J_c [2][BH][NC] (fp32, [n][j])
+  const float* S0f;      // [BH][d][d] or null (frames, chunks)
+  const float* S0r;
+  const float* alpha;    // [BH][T][d] or null (frames, compose)
+  float* states;         // frames, chunks: boundary states [2][BH][NC + 1]
+  float* Jout;           // compose: J_c [2][BH][NC]
+  uint8_t* Pout;         // compose: P_c images [2][BH][NC]
+  int BH, T, chunk, NC;
+};
+
 struct ScanCfg {
   static constexpr int THREADS = 320;
   static constexpr int PREFETCH = 3;                       // steps of L2 prefetch lead
@@ -793,10 +821,8 @@ __device__ __forceinline__ uint32_t ximg_offset(int n, int k) {
   return (uint32_t)(k >> 6) * 16384u + sw128_offset((uint32_t)n, (uint32_t)(k & 63));
 }
 
-__global__ void __launch_bounds__(ScanCfg::THREADS, 1)
-k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
-          const float* __restrict__ S0f, const float* __restrict__ S0r, const float* __restrict__ alpha,
-          float* __restrict__ states, int BH, int T, int chunk, int NC) {
+template <int MODE>
+__global__ void __launch_bounds__(ScanCfg::THREADS, 1) k_scan_tc(const ScanArgs sa) {
   using C = ScanCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -807,7 +833,31 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x, dir = blockIdx.y;
+  // composing: the four CTAs of a chunk (2 directions x 2 parts) are
+  // neighbours and share the chunk's M images and B through L2
+  const int dir = MODE == kScanCompose ? (int)((blockIdx.x >> 1) & 1u) : (int)blockIdx.y;
+  const int T = sa.T, NC = sa.NC, BH = sa.BH;
+  // chain (b, h) and, when composing, the chunk, its first frame, the part
+  // (0: J, 1: P) and the step count L
+  int bh, cc = 0, c0 = 0, part = 0, L;
+  if (MODE == kScanCompose) {
+    const int u = blockIdx.x;
+    part = u & 1;
+    bh = (u >> 2) / NC;
+    cc = (u >> 2) % NC;
+    c0 = cc * sa.chunk;
+    L = min(sa.chunk, T - c0);
+  } else {
+    bh = blockIdx.x;
+    L = MODE == kScanFrames ? T : NC;
+  }
+  const bool withB = !(MODE == kScanCompose && part == 1);
+  // operand index of step i: a frame (frames, compose) or a chunk map (chunks)
+  auto src_of = [&](int i) -> size_t {
+    if (MODE == kScanFrames) return (size_t)bh * T + (dir == 0 ? i : T - 1 - i);
+    if (MODE == kScanCompose) return (size_t)bh * T + c0 + (dir == 0 ? i : L - 1 - i);
+    return ((size_t)dir * BH + bh) * NC + (dir == 0 ? i : NC - 1 - i);
+  };
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(MFULL + s), 1);
@@ -826,25 +876,24 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  grid_wait_prerequisites();   // M images and B are complete (see k_stats_tc)
+  grid_wait_prerequisites();   // the operand images and B are complete (see k_stats_tc)
   grid_launch_dependents();
   const uint32_t tmem = *tmem_slot;
-  auto frame_of = [&](int i) { return dir == 0 ? i : T - 1 - i; };
   int last_i[2] = {-1, -1};   // producer: last step issued on each stage
 
   if (warp == C::WARP_PROD) {
-    // ---------------- M image producer
+    // ---------------- operand image producer
     if (lane == 0) {
-      for (int i = 0; i < T; ++i) {
+      for (int i = 0; i < L; ++i) {
         const uint32_t s = (uint32_t)i & 1u, ph = ((uint32_t)i >> 1) & 1u;
         if (!mbar_wait(BAR(MEMPTY + s), ph ^ 1u, abort_flag)) break;
         mbar_arrive_expect_tx(BAR(MFULL + s), kImgBytes);
-        const uint8_t* src = Mimg + ((size_t)bh * T + frame_of(i)) * kImgBytes;
+        const uint8_t* src = sa.Mimg + src_of(i) * kImgBytes;
         const uint32_t dst = sbase + C::OFF_M + s * kImgBytes;
-        if (i + C::PREFETCH < T) {   // warm L2 with the M image and B of a later step
-          const size_t fa = (size_t)bh * T + frame_of(i + C::PREFETCH);
-          bulk_prefetch_l2(Mimg + fa * kImgBytes, kImgBytes);
-          bulk_prefetch_l2(Bm + fa * kDD, (uint32_t)(kDD * sizeof(float)));
+        if (i + C::PREFETCH < L) {   // warm L2 with the image and B of a later step
+          const size_t fa = src_of(i + C::PREFETCH);
+          bulk_prefetch_l2(sa.Mimg + fa * kImgBytes, kImgBytes);
+          if (withB) bulk_prefetch_l2(sa.Bm + fa * kDD, (uint32_t)(kDD * sizeof(float)));
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) bulk_load(dst + q * 16384u, src + q * 16384u, 16384u, BAR(MFULL + s));
@@ -856,7 +905,7 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
     if (lane == 0) {
       constexpr uint32_t kId = idesc_bf16(128, 64, 1, 1);   // A (M image) and B (X half) MN-major
       bool ok = true;
-      for (int i = 0; ok && i < T; ++i) {
+      for (int i = 0; ok && i < L; ++i) {
         const uint32_t s = (uint32_t)i & 1u, ph = ((uint32_t)i >> 1) & 1u;
         if (!mbar_wait(BAR(MFULL + s), ph, abort_flag)) break;
         const uint32_t mh = sbase + C::OFF_M + s * kImgBytes, ml = mh + kImgHalf;
@@ -886,29 +935,37 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
     // ---------------- state warps: half h = warp / 4, thread j owns column j of S
     const int h = warp >> 2, q = warp & 3;
     const int j = q * 32 + lane;
-    const float* S0 = dir == 0 ? S0f : S0r;
-    float* st = states + ((size_t)dir * BH + bh) * (size_t)(NC + 1) * kDD;
+    const float* S0 = dir == 0 ? sa.S0f : sa.S0r;
+    float* st = MODE == kScanCompose ? nullptr
+                                     : sa.states + ((size_t)dir * BH + bh) * (size_t)(NC + 1) * kDD;
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + 64u * (uint32_t)h;
     // X image: row k = j, 16-B chunk c (n2 = 8c .. 8c+7) at ((c ^ (j & 7)) << 4)
-    const uint32_t xrow = sbase + C::OFF_X + (uint32_t)h * 2u * C::XIMG + (uint32_t)j * 128u;
+    const uint32_t xbase = sbase + C::OFF_X + (uint32_t)h * 2u * C::XIMG;
+    const uint32_t xrow = xbase + (uint32_t)j * 128u;
     const uint32_t jsw = (uint32_t)(j & 7);
     float bnext[64];
 
-    // initial state: store it as the first boundary, X_0 = S0 + B_{t0}
+    // initial state (stored as the first boundary) and X_0 = S0 Diag(alpha) + B
     {
       const int j0 = dir == 0 ? 0 : NC;
-      const float* B0 = Bm + ((size_t)bh * T + frame_of(0)) * kDD + (size_t)(64 * h) * kD + j;
+      const float* B0 = sa.Bm + src_of(0) * kDD + (size_t)(64 * h) * kD + j;
       // decay of the first frame on key column j (Eq. 2); 1 without decay
-      const float a0 = alpha ? __ldg(alpha + ((size_t)bh * T + frame_of(0)) * kD + j) : 1.f;
+      const float a0 = (MODE != kScanChunks && sa.alpha) ? __ldg(sa.alpha + src_of(0) * kD + j) : 1.f;
 #pragma unroll 2
       for (int c = 0; c < 8; ++c) {
         float x[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int n = 64 * h + 8 * c + e;
-          const float s0 = S0 ? __ldg(S0 + (size_t)bh * kDD + (size_t)n * kD + j) : 0.f;
-          st[(size_t)j0 * kDD + (size_t)n * kD + j] = s0;
-          x[e] = fmaf(s0, a0, __ldg(B0 + (size_t)(8 * c + e) * kD));
+          float s0;
+          if (MODE == kScanCompose) {
+            s0 = (part == 1 && n == j) ? 1.f : 0.f;
+          } else {
+            s0 = S0 ? __ldg(S0 + (size_t)bh * kDD + (size_t)n * kD + j) : 0.f;
+            st[(size_t)j0 * kDD + (size_t)n * kD + j] = s0;
+          }
+          if (MODE == kScanChunks) x[e] = s0;
+          else x[e] = fmaf(s0, a0, withB ? __ldg(B0 + (size_t)(8 * c + e) * kD) : 0.f);
         }
         const uint32_t o = xrow + (((uint32_t)c ^ jsw) << 4);
         st_chunk_hilo(o, o + C::XIMG, x);
@@ -916,22 +973,30 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
       fence_proxy_async_smem();
       mbar_arrive(BAR(XFULL + h));
     }
-    for (int i = 0; i < T; ++i) {
-      const bool more = i + 1 < T;
-      const int t = frame_of(i);
-      int jb = -1;
-      if (dir == 0) {
-        if ((t + 1) % chunk == 0 || t == T - 1) jb = (t + chunk) / chunk;
-      } else if (t % chunk == 0) {
-        jb = t / chunk;
+    for (int i = 0; i < L; ++i) {
+      const bool more = i + 1 < L;
+      int jb = -1;   // boundary state reached after this step
+      if (MODE == kScanFrames) {
+        const int t = dir == 0 ? i : T - 1 - i;
+        if (dir == 0) {
+          if ((t + 1) % sa.chunk == 0 || t == T - 1) jb = (t + sa.chunk) / sa.chunk;
+        } else if (t % sa.chunk == 0) {
+          jb = t / sa.chunk;
+        }
+      } else if (MODE == kScanChunks) {
+        const int c = dir == 0 ? i : NC - 1 - i;
+        jb = dir == 0 ? c + 1 : c;
       }
       float anext = 1.f;   // decay of the next frame on key column j (Eq. 2)
-      if (more) {   // B_{t+1}[64h + n2][j]: 32 lanes read 128 contiguous bytes per row
-        const float* Bn = Bm + ((size_t)bh * T + frame_of(i + 1)) * kDD + (size_t)(64 * h) * kD + j;
+      // B of the next frame, or this chunk's J: 32 lanes read 128 contiguous bytes per row
+      const bool loadB = MODE == kScanChunks || (more && withB);
+      if (loadB) {
+        const size_t si = MODE == kScanChunks ? src_of(i) : src_of(i + 1);
+        const float* Bn = sa.Bm + si * kDD + (size_t)(64 * h) * kD + j;
 #pragma unroll
         for (int n2 = 0; n2 < 64; ++n2) bnext[n2] = __ldg(Bn + (size_t)n2 * kD);
-        if (alpha) anext = __ldg(alpha + ((size_t)bh * T + frame_of(i + 1)) * kD + j);
       }
+      if (MODE != kScanChunks && more && sa.alpha) anext = __ldg(sa.alpha + src_of(i + 1) * kD + j);
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(DFULL + h), (uint32_t)i & 1u, abort_flag))) break;
       tc_fence_after();
 #pragma unroll
@@ -939,17 +1004,42 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
         uint32_t v[16];
         tmem_ld16(trow + cb * 16, v);
         tmem_wait_ld();
-        if (jb >= 0) {
+        float y[16];   // the state after this step
 #pragma unroll
-          for (int c = 0; c < 16; ++c) st[(size_t)jb * kDD + (size_t)(64 * h + cb * 16 + c) * kD + j] = __uint_as_float(v[c]);
+        for (int c = 0; c < 16; ++c)
+          y[c] = MODE == kScanChunks ? __uint_as_float(v[c]) + bnext[cb * 16 + c] : __uint_as_float(v[c]);
+        if (MODE != kScanCompose && jb >= 0) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) st[(size_t)jb * kDD + (size_t)(64 * h + cb * 16 + c) * kD + j] = y[c];
+        }
+        if (MODE == kScanCompose && !more) {
+          const size_t co = ((size_t)dir * BH + bh) * NC + cc;
+          if (part == 0) {   // J_c, fp32 [n][j]
+            float* jo = sa.Jout + co * kDD + (size_t)(64 * h + cb * 16) * kD + j;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) jo[(size_t)c * kD] = y[c];
+          } else {   // P_c as the operand image (element (j, n) = P[n][j]), this half's rows, in its X area
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const int nl = cb * 16 + c;   // row within the half
+              const float hi = __bfloat162float(__float2bfloat16_rn(y[c]));
+              const uint32_t off = (uint32_t)(j >> 6) * 8192u + sw128_offset((uint32_t)nl, (uint32_t)(j & 63));
+              st_shared_u16(xbase + off, __bfloat16_as_ushort(__float2bfloat16_rn(y[c])));
+              st_shared_u16(xbase + 16384u + off, __bfloat16_as_ushort(__float2bfloat16_rn(y[c] - hi)));
+            }
+          }
         }
         if (more) {
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
+          for (int q2 = 0; q2 < 2; ++q2) {
             float x[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = fmaf(__uint_as_float(v[8 * q + e]), anext, bnext[cb * 16 + 8 * q + e]);
-            const uint32_t c8 = (uint32_t)(2 * cb + q);
+            for (int e = 0; e < 8; ++e) {
+              const int c = 8 * q2 + e;
+              x[e] = MODE == kScanChunks ? y[c]
+                                         : fmaf(y[c], anext, withB ? bnext[cb * 16 + c] : 0.f);
+            }
+            const uint32_t c8 = (uint32_t)(2 * cb + q2);
             const uint32_t o = xrow + ((c8 ^ jsw) << 4);
             st_chunk_hilo(o, o + C::XIMG, x);
           }
@@ -959,6 +1049,21 @@ k_scan_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bm,
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(BAR(XFULL + h));
+      }
+    }
+    if (MODE == kScanCompose && part == 1) {
+      // this half's rows of the P_c image: 4 pieces of 8 KB (hi / lo x two
+      // 64-column blocks) -> global, 16 B per thread per copy
+      named_bar_sync(1u + (uint32_t)h, 128);
+      uint8_t* img = sa.Pout + (((size_t)dir * BH + bh) * NC + cc) * kImgBytes;
+      const int t = q * 32 + lane;
+#pragma unroll 4
+      for (int k2 = 0; k2 < 16; ++k2) {
+        const uint32_t o = 16u * (uint32_t)(t + 128 * k2);
+        const uint32_t piece = o >> 13, within = o & 8191u;
+        const uint4 val = ld_shared_v4(xbase + o);
+        *reinterpret_cast<uint4*>(img + (size_t)(piece >> 1) * kImgHalf + (size_t)(piece & 1u) * 16384u +
+                                  8192u * (uint32_t)h + within) = val;
       }
     }
   }
@@ -1479,15 +1584,46 @@ inline int launch_inverse(const float* A, size_t FH, uint8_t* Mimg, float* M_dbg
                     Mimg, M_dbg);
 }
 
+template <int MODE>
+inline int launch_scan_mode(const ScanArgs& sa, dim3 grid, cudaStream_t s) {
+  if (cudaFuncSetAttribute(k_scan_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanCfg::SMEM) !=
+      cudaSuccess)
+    return VDA_ERR_CUDA;
+  const char* name = MODE == kScanFrames ? "k_scan_tc<frames>"
+                                         : (MODE == kScanCompose ? "k_scan_tc<compose>" : "k_scan_tc<chunks>");
+  return launch_pdl(name, k_scan_tc<MODE>, grid, dim3(ScanCfg::THREADS), ScanCfg::SMEM, s, sa);
+}
+
+// Per-frame scans: one CTA per (b, h, direction), T steps.
 inline int launch_scan(const uint8_t* Mimg, const float* Bm, const float* S0f, const float* S0r,
                        const float* alpha, float* states, size_t BH, int T, int chunk, int NC, int ndir,
                        cudaStream_t s) {
-  if (cudaFuncSetAttribute(k_scan_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ScanCfg::SMEM) !=
-      cudaSuccess)
-    return VDA_ERR_CUDA;
-  dim3 grid((unsigned)BH, (unsigned)ndir);
-  return launch_pdl("k_scan_tc", k_scan_tc, grid, dim3(ScanCfg::THREADS), ScanCfg::SMEM, s, Mimg, Bm, S0f, S0r,
-                    alpha, states, (int)BH, T, chunk, NC);
+  const ScanArgs sa{Mimg, Bm, S0f, S0r, alpha, states, nullptr, nullptr, (int)BH, T, chunk, NC};
+  return launch_scan_mode<kScanFrames>(sa, dim3((unsigned)BH, (unsigned)ndir), s);
+}
+
+// Bytes of the chunk maps of the chunk-wise scans: J_c (fp32) and the P_c
+// operand image for every (direction, b, h, chunk).
+inline size_t chunk_maps_bytes(size_t BH, int NC) {
+  return 2 * BH * (size_t)NC * (kDD * sizeof(float) + kImgBytes);
+}
+
+// Chunk-wise scans: compose every chunk's maps (2 x 2 x BH x NC CTAs of at
+// most `chunk` steps), then scan the NC maps per chain.  `maps` holds
+// chunk_maps_bytes(BH, NC) bytes, 256-B aligned.
+template <typename Timer>
+inline int launch_scan_chunked(const uint8_t* Mimg, const float* Bm, const float* S0f, const float* S0r,
+                               const float* alpha, float* states, char* maps, size_t BH, int T, int chunk,
+                               int NC, cudaStream_t s, Timer& timer) {
+  float* J = reinterpret_cast<float*>(maps);
+  uint8_t* P = reinterpret_cast<uint8_t*>(maps + 2 * BH * (size_t)NC * kDD * sizeof(float));
+  const ScanArgs comp{Mimg, Bm, nullptr, nullptr, alpha, nullptr, J, P, (int)BH, T, chunk, NC};
+  int rc = launch_scan_mode<kScanCompose>(comp, dim3((unsigned)(4 * BH * (size_t)NC)), s);
+  if (rc != VDA_OK) return rc;
+  timer.end(2, s);
+  timer.begin(2, s);
+  const ScanArgs chains{P, J, S0f, S0r, nullptr, states, nullptr, nullptr, (int)BH, T, chunk, NC};
+  return launch_scan_mode<kScanChunks>(chains, dim3((unsigned)BH, 2u), s);
 }
 
 inline int launch_readout(const void* Q, const void* G, const float* w, const float* states, const float* bridge,
@@ -1533,7 +1669,21 @@ inline size_t tc_extra_workspace_bytes(bool tc, size_t FH, int d) {
   return tc ? FH * (size_t)tc::kImgBytes : 0;
 }
 
-inline int tc_launches_per_forward() { return 4; }
+// Scan form of the tensor-core path.  Automatic choice: the chunk-wise scans
+// when their composition CTAs (4 per (b, h) and chunk) fill the GPU in at
+// most two waves (few (b, h) pairs: the per-frame chains would leave most SMs
+// idle for T steps), else the per-frame scans.
+inline bool use_chunk_scan(int form, size_t BH, int T, int chunk, int NC, int sms) {
+  if (form == VDA_SCAN_FRAMES) return false;
+  if (form == VDA_SCAN_CHUNKS) return true;
+  return chunk > 1 && T > chunk && 4 * BH * (size_t)NC <= 2 * (size_t)sms;
+}
+
+// Kernel launches of one forward on the tensor-core path (without the decay
+// bridge): the chunk-wise scans take two.
+inline int tc_launches_per_forward(int form, size_t BH, int T, int chunk, int NC) {
+  return use_chunk_scan(form, BH, T, chunk, NC, tc::num_sms()) ? 5 : 4;
+}
 
 // The launch schedule on the caller's stream: Gram kernel, inverse, scan,
 // decay bridge (with a decay gate), readout.  Timer hooks begin(stage, stream)
@@ -1541,8 +1691,8 @@ inline int tc_launches_per_forward() { return 4; }
 // 3 readout).
 template <typename Timer>
 int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_args& a, char* ws_AM,
-              char* ws_B, char* ws_states, char* ws_img, char* ws_bridge, cudaStream_t s, float* stats_out,
-              Timer& timer) {
+              char* ws_B, char* ws_states, char* ws_img, char* ws_bridge, char* ws_maps, cudaStream_t s,
+              float* stats_out, Timer& timer) {
   const size_t FH = BH * (size_t)T;
   const size_t fdd = FH * tc::kDD;
   float* A = reinterpret_cast<float*>(ws_AM);
@@ -1563,8 +1713,11 @@ int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_
   timer.end(1, s);
   if ((rc = debug_check("inverse", s)) != VDA_OK) return rc;
   timer.begin(2, s);
-  if ((rc = tc::launch_scan(img, Bt, a.S0_fwd, a.S0_rev, a.alpha, st, BH, T, chunk, NC, 2, s)) != VDA_OK)
-    return rc;
+  if (use_chunk_scan(a.scan_form, BH, T, chunk, NC, tc::num_sms()))
+    rc = tc::launch_scan_chunked(img, Bt, a.S0_fwd, a.S0_rev, a.alpha, st, ws_maps, BH, T, chunk, NC, s, timer);
+  else
+    rc = tc::launch_scan(img, Bt, a.S0_fwd, a.S0_rev, a.alpha, st, BH, T, chunk, NC, 2, s);
+  if (rc != VDA_OK) return rc;
   timer.end(2, s);
   if ((rc = debug_check("scan", s)) != VDA_OK) return rc;
   float* bridge = nullptr;

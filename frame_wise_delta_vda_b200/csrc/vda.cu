@@ -36,7 +36,7 @@ struct Plan {
   int B, H, T, U, d, chunk, window, NC, dtype;
   size_t BH, FH;
   bool tc;               // tensor-core (tcgen05) kernels
-  size_t off_AM, off_B, off_states, off_bridge, total;
+  size_t off_AM, off_B, off_states, off_bridge, off_maps, total;
 };
 
 int check_sizes(int B, int H, int T, int U, int d_k, int d_v, int chunk, int window, int dtype) {
@@ -66,6 +66,16 @@ Plan make_plan(int B, int H, int T, int U, int d, int chunk, int window, int dty
   p.off_B = off;      off = align_up(off + p.FH * dd);
   p.off_states = off; off = align_up(off + 2 * p.BH * (size_t)(p.NC + 1) * dd);
   p.off_bridge = off; off = align_up(off + 2 * p.FH * (size_t)d * sizeof(float));   // decay bridge products
+  // chunk maps of the chunk-wise scans (tensor-core path): in A's region,
+  // which the scans no longer need, when they fit there
+  p.off_maps = p.off_AM;
+  if (p.tc) {
+    const size_t maps = vda::tc::chunk_maps_bytes(p.BH, p.NC);
+    if (maps > p.FH * dd) {
+      p.off_maps = off;
+      off = align_up(off + maps);
+    }
+  }
   p.total = off + vda::tc_extra_workspace_bytes(p.tc, p.FH, d);
   return p;
 }
@@ -209,6 +219,7 @@ int validate_args(const vda_args* a) {
   if ((a->S0_fwd && !aligned16(a->S0_fwd)) || (a->S0_rev && !aligned16(a->S0_rev)) ||
       (a->alpha && !aligned16(a->alpha)))
     return VDA_ERR_INVALID_ARGUMENT;
+  if (a->scan_form < VDA_SCAN_AUTO || a->scan_form > VDA_SCAN_CHUNKS) return VDA_ERR_INVALID_ARGUMENT;
   return VDA_OK;
 }
 
@@ -220,7 +231,7 @@ int forward_impl(const vda_args& a, char* ws, const Plan& p, float* states_out, 
   if (p.tc) {
     rc = vda::launch_tc(p.BH, p.T, p.U, p.chunk, p.NC, p.window, a, ws + p.off_AM, ws + p.off_B,
                         ws + p.off_states, ws + p.total - vda::tc_extra_workspace_bytes(true, p.FH, p.d),
-                        ws + p.off_bridge, s, stats_out, tm);
+                        ws + p.off_bridge, ws + p.off_maps, s, stats_out, tm);
   } else if (p.dtype == VDA_BF16) {
     rc = dispatch_simt<__nv_bfloat16>(p, a, ws, s, tm, stats_out);
   } else {
@@ -429,7 +440,7 @@ size_t vda_workspace_bytes(int B, int H, int T, int U, int d_k, int d_v, int chu
 int vda_launches_per_forward(int B, int H, int T, int U, int d_k, int d_v, int chunk, int dtype) {
   if (check_sizes(B, H, T, U, d_k, d_v, chunk, 0, dtype) != VDA_OK) return 0;
   const Plan p = make_plan(B, H, T, U, d_k, chunk, 0, dtype);
-  return p.tc ? vda::tc_launches_per_forward() : 4;
+  return p.tc ? vda::tc_launches_per_forward(VDA_SCAN_AUTO, p.BH, p.T, p.chunk, p.NC) : 4;
 }
 
 int vda_forward_ex(const vda_args* args, void* workspace, size_t workspace_bytes,

@@ -83,6 +83,23 @@ typedef enum vda_dtype {
   VDA_F32 = 1   /* ... are float32 */
 } vda_dtype;
 
+/* How the forward and reverse scans of Section 2.2 run on the tensor-core
+ * path (d = 128, bf16); the SIMT path always scans frame by frame.  Both give
+ * the same boundary states up to rounding.
+ *   VDA_SCAN_FRAMES: one sequential chain of T frame updates per (b, h,
+ *     direction), S <- (S Diag(alpha_t) + B_t) M_t.
+ *   VDA_SCAN_CHUNKS: the chunk-wise scan of Section 5 ("Chunk-wise scans",
+ *     Appendix A.1): every chunk's frames are first composed, in parallel,
+ *     into one affine map S -> S P_c + J_c, then each chain runs its NC maps.
+ *     About twice the tensor-core work on a chain of chunk + NC steps; it pays
+ *     when few (b, h) pairs share the GPU.
+ *   VDA_SCAN_AUTO: the library picks by the number of (b, h) pairs. */
+typedef enum vda_scan_form {
+  VDA_SCAN_AUTO = 0,
+  VDA_SCAN_FRAMES = 1,
+  VDA_SCAN_CHUNKS = 2
+} vda_scan_form;
+
 /* Full argument block of vda_forward_ex. */
 typedef struct vda_args {
   int dtype;                  /* vda_dtype of q, k, v, gate, out */
@@ -101,6 +118,7 @@ typedef struct vda_args {
   float eps;                  /* RMSNorm epsilon; <= 0 selects 1e-6 */
   void* stream;               /* cudaStream_t */
   const float* alpha;         /* [B,H,T,d_k] decay gates in [0,1] (Eq. 2), or NULL: no decay */
+  int scan_form;              /* vda_scan_form; 0 (zero-initialised args) = VDA_SCAN_AUTO */
 } vda_args;
 
 /* Bidirectional VDA forward, bf16 I/O.  Takes its workspace stream-ordered
@@ -211,8 +229,9 @@ VDA_API int vda_timing_enable(int max_calls);
 VDA_API int vda_timing_read(float* stage_ms, int n_stages, int* calls);
 
 /* Number of kernel launches one vda_forward_ex call with these sizes makes
- * without a decay gate; with vda_args.alpha set the call makes one more (the
- * bridge products of Eq. A.4). */
+ * without a decay gate and with scan_form VDA_SCAN_AUTO on the current device
+ * (the chunk-wise scans take two launches); with vda_args.alpha set the call
+ * makes one more (the bridge products of Eq. A.4). */
 VDA_API int vda_launches_per_forward(int B, int H, int T, int U, int d_k, int d_v, int chunk, int dtype);
 
 /* ---------------------------------------------------------------------------

@@ -74,6 +74,7 @@ def _args(**kw):
     (dict(dtype=3), 1),
     (dict(d_k=16, d_v=32), 2),             # d_k != d_v
     (dict(d_k=48, d_v=48), 2),             # unsupported head dim
+    (dict(scan_form=3), 1), (dict(scan_form=-1), 1),
 ])
 def test_forward_ex_rejects_bad_arguments(L, kw, status):
     a = _args(**kw)
@@ -104,6 +105,22 @@ def test_text_state_and_host_entry_validation(L):
 def test_launch_count(L):
     assert L.vda_launches_per_forward(1, 2, 10, 16, 16, 16, 5, 1) >= 4
     assert L.vda_launches_per_forward(1, 2, 10, 16, 16, 24, 5, 1) == 0
+    # tensor-core path: per-frame scans at 48 heads (4 launches), chunk-wise
+    # scans (compose + chunk chains: 5 launches) at 6 heads of the same shapes;
+    # without a GPU the library assumes 148 SMs
+    assert L.vda_launches_per_forward(1, 48, 60, 1008, 128, 128, 5, 0) == 4
+    assert L.vda_launches_per_forward(1, 6, 60, 1008, 128, 128, 5, 0) == 5
+    assert L.vda_launches_per_forward(1, 6, 60, 1008, 128, 128, 1, 0) == 4   # one-frame chunks
+
+
+def test_chunk_maps_fit_the_workspace(L):
+    # the chunk maps (J_c fp32 + P_c image, 128 KB per direction and chunk)
+    # live in A's region when 4 NC <= T, else in a region of their own
+    fh_dd = 128 * 128 * 4
+    base = L.vda_workspace_bytes(1, 6, 60, 1008, 128, 128, 5, 0)
+    one = L.vda_workspace_bytes(1, 6, 60, 1008, 128, 128, 1, 0)
+    assert one - base >= 2 * 6 * (60 - 12) * fh_dd       # more boundary states and the maps
+    assert one >= 6 * 60 * fh_dd + 4 * 6 * 60 * fh_dd
 
 
 def test_timing_read_without_calls(L):
