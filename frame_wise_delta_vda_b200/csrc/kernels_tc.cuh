@@ -33,6 +33,11 @@ constexpr int kD = 128;
 constexpr size_t kDD = (size_t)kD * kD;
 constexpr uint32_t kImgHalf = 32768;   // one bf16 128x128 operand image
 constexpr uint32_t kImgBytes = 65536;  // hi + lo images
+// A_t is symmetric, so the Gram kernel stores its upper block triangle only:
+// 16 x 16 blocks (br, bc) with br <= bc, block (br, bc) at
+// (bc (bc + 1) / 2 + br) * 256 floats, element (r, c) of a block at c * 16 + r.
+constexpr size_t kATri = 36 * 256;      // floats per frame-head
+__host__ __device__ constexpr size_t atri_block(int br, int bc) { return (size_t)((bc * (bc + 1)) / 2 + br) * 256; }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -47,7 +52,8 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 // 64 channels x 64 tokens lands as 64 rows of 128 B with the 128-B swizzle.
 //
 // Persistent CTAs (one per SM) walk frame-heads fh = blockIdx.x + i*grid.
-// Warps: 0-3 epilogue (TMEM -> A and B, fp32, standard layouts, coalesced),
+// Warps: 0-3 epilogue (TMEM -> A (upper block triangle) and B, fp32,
+//        coalesced; optionally the full A for the debug output),
 //        4-11 scale (beta*K hi/lo), 12 TMA producer, 13 MMA issuer + TMEM
 //        owner.  Two TMEM accumulators: the epilogue of one frame-head
 //        overlaps the MMAs of the next.
@@ -121,7 +127,7 @@ __device__ __forceinline__ void store_img_chunk(uint8_t* img, uint32_t off, cons
 __global__ void __launch_bounds__(StatsCfg::THREADS, 1)
 k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
            const float* __restrict__ beta, int U, int FH, float* __restrict__ A_out,
-           float* __restrict__ B_out) {
+           float* __restrict__ B_out, float* __restrict__ A_full) {
   using C = StatsCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -282,8 +288,11 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
     }
   } else {
     // ---------------- epilogue: TMEM lane i = row i of D; column c of D goes to
-    // A[c][i] (A is symmetric) or B[c - 128][i]: 32 lanes store 128 contiguous bytes
+    // element (i, c) of A's block (i / 16, c / 16) when that block is in the
+    // upper triangle (16 lanes store 64 contiguous bytes), or B[c - 128][i]
+    // (32 lanes store 128 contiguous bytes)
     const int i = warp * 32 + lane;
+    const int br = i >> 4;
     const uint32_t lb = (uint32_t)(warp * 32) << 16;
     uint32_t lf = 0;
     for (int fh = blockIdx.x; fh < FH; fh += gridDim.x, ++lf) {
@@ -291,7 +300,7 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(TFULL + buf), bph, abort_flag))) break;
       tc_fence_after();
       const uint32_t tA = tmem + buf * 256u;
-      float* Af = A_out + (size_t)fh * kDD;
+      float* At = A_out + (size_t)fh * kATri + (i & 15);
       float* Bf = B_out + (size_t)fh * kDD;
 #pragma unroll 1
       for (int q = 0; q < 8; ++q) {
@@ -302,9 +311,26 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
           tc_fence_before();
           mbar_arrive(BAR(TEMPTY + buf));
         }
-        float* dst = q < 4 ? Af + (size_t)(32 * q) * kD : Bf + (size_t)(32 * (q - 4)) * kD;
+        if (q < 4) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) dst[(size_t)c * kD + i] = __uint_as_float(v0[c]);
+          for (int hb = 0; hb < 2; ++hb) {
+            const int bc = 2 * q + hb;
+            if (bc >= br) {
+              float* dst = At + atri_block(br, bc);
+#pragma unroll
+              for (int c = 0; c < 16; ++c) dst[16 * c] = __uint_as_float(v0[16 * hb + c]);
+            }
+          }
+          if (A_full) {   // debug output: the full matrix
+            float* dst = A_full + (size_t)fh * kDD + (size_t)(32 * q) * kD + i;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) dst[(size_t)c * kD] = __uint_as_float(v0[c]);
+          }
+        } else {
+          float* dst = Bf + (size_t)(32 * (q - 4)) * kD + i;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) dst[(size_t)c * kD] = __uint_as_float(v0[c]);
+        }
       }
     }
   }
@@ -349,7 +375,7 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
 // date in fp32 (A_QQ + X_Q C_Q^T) and sweeps it while the tensor cores apply
 // the update.  Four warpgroups per CTA work on four matrices at once (own
 // TMEM columns, shared-memory workspace, named barriers, completion barriers).
-// In: A rows (fp32, from k_stats_tc).  Out: the scan's M operand image
+// In: A (fp32, upper block triangle, from k_stats_tc).  Out: the scan's M operand image
 // (element (j, k) = M[k][j], MN-major, 128-B swizzle, bf16 hi / lo halves)
 // and optionally M in fp32.
 // ===========================================================================
@@ -642,6 +668,42 @@ __device__ __forceinline__ bool sweep_inverse_tmem(uint32_t tA, uint32_t lb, uin
   return ok;
 }
 
+// Row i, columns [64 hh, 64 hh + 64) of a symmetric A stored as its upper
+// block triangle (kATri layout): blocks at or right of the diagonal give the
+// row directly (16 lanes of a row block read 64 contiguous bytes per column),
+// blocks left of it give the transposed block's column, contiguous per thread.
+__device__ __forceinline__ void load_a_row_half(const float* __restrict__ At, int i, int hh, float (&a)[64]) {
+  const int br = i >> 4, r = i & 15;
+#pragma unroll
+  for (int b4 = 0; b4 < 4; ++b4) {
+    const int bc = 4 * hh + b4;
+    if (bc >= br) {
+      const float* blk = At + atri_block(br, bc) + r;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) a[16 * b4 + c] = __ldg(blk + 16 * c);
+    } else {
+      const float4* blk = reinterpret_cast<const float4*>(At + atri_block(bc, br) + 16 * r);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float4 x = __ldg(blk + c);
+        a[16 * b4 + 4 * c] = x.x; a[16 * b4 + 4 * c + 1] = x.y;
+        a[16 * b4 + 4 * c + 2] = x.z; a[16 * b4 + 4 * c + 3] = x.w;
+      }
+    }
+  }
+}
+
+// 64 fp32 values -> TMEM lane columns [col, col + 64)
+__device__ __forceinline__ void tmem_st64f(uint32_t taddr, const float (&a)[64]) {
+  uint32_t w[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(a[c]);
+  tmem_st32(taddr, w);
+#pragma unroll
+  for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(a[32 + c]);
+  tmem_st32(taddr + 32u, w);
+}
+
 __global__ void __launch_bounds__(InvCfg::THREADS, 1)
 k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, float* __restrict__ M_dbg) {
   using C = InvCfg;
@@ -676,52 +738,55 @@ k_inverse_tc(const float* __restrict__ A, int FH, uint8_t* __restrict__ Mimg, fl
                      sbase + C::BAR_OFF + 8u * (uint32_t)(C::GROUPS + g)};
   uint32_t sphase = 0, xphase = 0;
 
-  for (int m = blockIdx.x * C::GROUPS + g; m < FH; m += gridDim.x * C::GROUPS) {
-    // row i of A -> TMEM lane i
-    const float4* Ar = reinterpret_cast<const float4*>(A + (size_t)m * kDD + (size_t)i * kD);
+  const int mstride = gridDim.x * C::GROUPS;
+  int m = blockIdx.x * C::GROUPS + g;
+  if (m < FH) {   // row i of the group's first matrix -> TMEM lane i
 #pragma unroll 1
-    for (int q = 0; q < 4; q += 2) {
-      uint32_t v[32], w[32];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float4 x = __ldg(Ar + 8 * q + c), y = __ldg(Ar + 8 * q + 8 + c);
-        v[4 * c] = __float_as_uint(x.x); v[4 * c + 1] = __float_as_uint(x.y);
-        v[4 * c + 2] = __float_as_uint(x.z); v[4 * c + 3] = __float_as_uint(x.w);
-        w[4 * c] = __float_as_uint(y.x); w[4 * c + 1] = __float_as_uint(y.y);
-        w[4 * c + 2] = __float_as_uint(y.z); w[4 * c + 3] = __float_as_uint(y.w);
-      }
-      tmem_st32(lb + tA + 32u * q, v);
-      tmem_st32(lb + tA + 32u * (q + 1), w);
+    for (int hh = 0; hh < 2; ++hh) {
+      float a[64];
+      load_a_row_half(A + (size_t)m * kATri, i, hh, a);
+      tmem_st64f(lb + tA + 64u * hh, a);
     }
-    const int mnext = m + gridDim.x * C::GROUPS;
-    if (i == 0 && mnext < FH)   // the group's next matrix: into L2 while this one is swept
-      bulk_prefetch_l2(A + (size_t)mnext * kDD, (uint32_t)(kDD * sizeof(float)));
+  }
+  for (; m < FH; m += mstride) {
+    const int mnext = m + mstride;
+    const bool has_next = mnext < FH;
+    if (i == 0 && has_next)   // the group's next matrix: into L2 while this one is swept
+      bulk_prefetch_l2(A + (size_t)mnext * kATri, (uint32_t)(kATri * sizeof(float)));
     tmem_wait_st();
     tc_fence_before();
     named_bar_sync(bid, 128);
     tc_fence_after();
     const bool ok = sweep_inverse_tmem(tA, lb, swb, bars, sphase, xphase, abort_flag, i, gw, lane, g, m & 3);
-    // M = -(swept matrix): row i -> operand image row i (k index), debug copy
+    // M = -(swept matrix): row i -> operand image row i (k index), debug copy.
+    // The next matrix's row i replaces each 64-column half once it has been
+    // read (this thread's own TMEM lane), so its loads overlap these stores.
     uint8_t* img = Mimg + (size_t)m * kImgBytes;
+    const float* An = A + (size_t)(has_next ? mnext : m) * kATri;
 #pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
-      uint32_t v[32];
-      tmem_ld32(lb + tA + 32u * q, v);
-      tmem_wait_ld();
+    for (int hh = 0; hh < 2; ++hh) {
+      float an[64];
+      if (has_next) load_a_row_half(An, i, hh, an);
+#pragma unroll 1
+      for (int q = 4 * hh; q < 4 * hh + 4; ++q) {   // 16-column slices
+        uint32_t v[16];
+        tmem_ld16(lb + tA + 16u * q, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float x[8];
+        for (int cc = 0; cc < 2; ++cc) {
+          float x[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = -__uint_as_float(v[8 * cc + e]);
-        store_img_chunk(img, mimg_offset(32 * q + 8 * cc, i), x);
+          for (int e = 0; e < 8; ++e) x[e] = -__uint_as_float(v[8 * cc + e]);
+          store_img_chunk(img, mimg_offset(16 * q + 8 * cc, i), x);
+        }
+        if (M_dbg) {
+          float* md = M_dbg + (size_t)m * kDD + (size_t)i * kD + 16 * q;
+#pragma unroll
+          for (int c2 = 0; c2 < 16; ++c2) md[c2] = -__uint_as_float(v[c2]);
+        }
       }
-      if (M_dbg) {
-        float* md = M_dbg + (size_t)m * kDD + (size_t)i * kD + 32 * q;
-#pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) md[c2] = -__uint_as_float(v[c2]);
-      }
+      if (has_next) tmem_st64f(lb + tA + 64u * hh, an);
     }
-    // the next matrix overwrites these TMEM rows: every lane's reads first
     tc_fence_before();
     const bool all_ok = named_bar_and(bid, 128, ok);
     tc_fence_after();
@@ -1556,7 +1621,7 @@ inline int num_sms() {
 // Statistics for FH frame-heads of U tokens (K, V: [FH][U][128] bf16):
 // A [FH][d_k][d_k] and B [FH][d_v][d_k], fp32.
 inline int launch_stats(const void* K, const void* V, const float* beta, int U, size_t FH, float* A, float* B,
-                        cudaStream_t s) {
+                        float* A_full, cudaStream_t s) {
   CUtensorMap tmK, tmV;
   if (!encode_bf16_3d(&tmK, K, (uint64_t)U, FH, 64) || !encode_bf16_3d(&tmV, V, (uint64_t)U, FH, 64))
     return VDA_ERR_CUDA;
@@ -1570,7 +1635,7 @@ inline int launch_stats(const void* K, const void* V, const float* beta, int U, 
   const size_t rounds = (FH + sms - 1) / sms;
   const int grid = (int)((FH + rounds - 1) / rounds);
   return launch_pdl("k_stats_tc", k_stats_tc, dim3(grid), dim3(StatsCfg::THREADS), StatsCfg::SMEM, s, tmK, tmV, beta,
-                    U, (int)FH, A, B);
+                    U, (int)FH, A, B, A_full);
 }
 
 // M = (I + A)^{-1} images (and optional fp32 copy) for FH matrices
@@ -1701,12 +1766,11 @@ int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_
   uint8_t* img = reinterpret_cast<uint8_t*>(ws_img);
   int rc;
   timer.begin(0, s);
-  if ((rc = tc::launch_stats(a.k, a.v, a.beta, U, FH, A, Bt, s)) != VDA_OK) return rc;
+  if ((rc = tc::launch_stats(a.k, a.v, a.beta, U, FH, A, Bt, stats_out, s)) != VDA_OK) return rc;
   timer.end(0, s);
   if ((rc = debug_check("stats", s)) != VDA_OK) return rc;
-  if (stats_out &&
-      (cudaMemcpyAsync(stats_out, A, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
-       cudaMemcpyAsync(stats_out + fdd, Bt, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess))
+  if (stats_out &&   // (the Gram kernel wrote the full A there)
+      cudaMemcpyAsync(stats_out + fdd, Bt, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
     return VDA_ERR_CUDA;
   timer.begin(1, s);
   if ((rc = tc::launch_inverse(A, FH, img, stats_out ? stats_out + 2 * fdd : nullptr, s)) != VDA_OK) return rc;
@@ -1744,7 +1808,7 @@ inline int tc_text_state(size_t BH, int L, const void* k, const void* v, const f
   float* Bt = reinterpret_cast<float*>(ws_B);
   uint8_t* img = reinterpret_cast<uint8_t*>(ws_img);
   int rc;
-  if ((rc = tc::launch_stats(k, v, beta, L, BH, A, Bt, s)) != VDA_OK) return rc;
+  if ((rc = tc::launch_stats(k, v, beta, L, BH, A, Bt, nullptr, s)) != VDA_OK) return rc;
   if ((rc = tc::launch_inverse(A, BH, img, nullptr, s)) != VDA_OK) return rc;
   return tc::launch_scan(img, Bt, nullptr, nullptr, nullptr, reinterpret_cast<float*>(ws_states), BH, 1, 1, 1, 1,
                          s);
