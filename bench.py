@@ -177,7 +177,8 @@ def algorithmic(wl):
 def stage_kernels(wl):
     """(limiter, kernel name, source files) of each stage's kernel on the path
     the library takes for this workload: tensor cores for bf16 I/O at
-    d_k = d_v = 128, the SIMT kernels otherwise.  The limiter is what sets the
+    d_k = d_v = 128 and 64 (at 64 with the FP32 Gauss-Jordan inverse), the
+    SIMT kernels otherwise.  The limiter is what sets the
     kernel's pace: "hbm" (streams its bytes near the copy bandwidth),
     "latency" (a dependent chain of small steps; its bytes are still measured
     against the HBM roofline) or "alu" (FP32 arithmetic)."""
@@ -185,6 +186,10 @@ def stage_kernels(wl):
         src = ["kernels_tc.cuh", "tc_ptx.cuh"]
         return {"stats": ("hbm", "k_stats_tc", src), "inverse": ("latency", "k_inverse_tc", src),
                 "scan": ("latency", "k_scan_tc", src), "readout": ("hbm", "k_readout_tc", src)}
+    if wl.dtype == "bf16" and wl.d == 64:
+        src = ["kernels_tc.cuh", "tc_ptx.cuh"]
+        return {"stats": ("hbm", "k_stats64_tc", src), "inverse": ("alu", "k_gj_inverse", ["kernels_simt.cuh"]),
+                "scan": ("latency", "k_scan64_tc", src), "readout": ("hbm", "k_readout_tc", src)}
     src = ["kernels_simt.cuh"]
     return {"stats": ("hbm", "k_stats_simt", src), "inverse": ("alu", "k_gj_inverse", src),
             "scan": ("latency", "k_scan_simt", src), "readout": ("hbm", "k_readout_simt", src)}

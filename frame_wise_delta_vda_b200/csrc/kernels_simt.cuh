@@ -1,8 +1,8 @@
 // kernels_simt.cuh - FP32 SIMT kernels of the VDA path.
 //
-// These serve the float32-I/O specialisation and the head dims below 128
-// (d in {16, 32, 64}); the bf16, d = 128 path uses the tcgen05 kernels.
-// The small-matrix inverse here is the FP32 path for every size.
+// These serve the float32-I/O specialisation and the head dims 16 and 32;
+// bf16 at d = 128 and d = 64 uses the tcgen05 kernels.  The small-matrix
+// inverse here is the FP32 path for every size but d = 128 with bf16.
 //
 // Paper: "Video DeltaNet" (arXiv 2609.20744): Eq. 3b (frame statistics),
 // Eq. 5 / Appendix A.1 (M_t = (I + A_t)^{-1}, S_t = (S_{t-1} + B_t) M_t),
@@ -94,10 +94,13 @@ k_stats_simt(const TIn* __restrict__ K, const TIn* __restrict__ V,
 // lives in registers: 16 x 16 threads, each holding a (D/16) x (D/16) block;
 // the pivot row and column are broadcast through double-buffered shared
 // memory, one barrier per elimination step.
+// With `img` (d = 64, the tensor-core scan) M is also written as that scan's
+// operand image: element (j, k) = M[k][j] in row k of 64 bf16 (128 B, 128-B
+// swizzle), hi part then lo part (8 KB each) per frame-head.
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256)
-k_gj_inverse(float* __restrict__ AM) {
+k_gj_inverse(float* __restrict__ AM, uint8_t* __restrict__ img) {
   constexpr int BS = D / 16;
   __shared__ float s_row[2][D];
   __shared__ float s_col[2][D];
@@ -153,6 +156,24 @@ k_gj_inverse(float* __restrict__ AM) {
   for (int i = 0; i < BS; ++i)
 #pragma unroll
     for (int j = 0; j < BS; ++j) Mx[(size_t)(r0 + i) * D + c0 + j] = a[i][j];
+  if constexpr (D == 64) {
+    if (img) {   // row k = r0 + i holds M[k][c0 .. c0 + 3]: 8 contiguous bytes of one 16-B chunk
+      uint8_t* dst = img + (size_t)blockIdx.x * 16384;
+#pragma unroll
+      for (int i = 0; i < BS; ++i) {
+        const uint32_t k = (uint32_t)(r0 + i);
+        const uint32_t off = k * 128u + (((((uint32_t)c0 >> 3) ^ (k & 7u)) & 7u) << 4) + (((uint32_t)c0 & 7u) << 1);
+        __nv_bfloat162 h01 = __floats2bfloat162_rn(a[i][0], a[i][1]), h23 = __floats2bfloat162_rn(a[i][2], a[i][3]);
+        const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+        __nv_bfloat162 l01 = __floats2bfloat162_rn(a[i][0] - f01.x, a[i][1] - f01.y);
+        __nv_bfloat162 l23 = __floats2bfloat162_rn(a[i][2] - f23.x, a[i][3] - f23.y);
+        *reinterpret_cast<uint2*>(dst + off) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&h01), *reinterpret_cast<uint32_t*>(&h23));
+        *reinterpret_cast<uint2*>(dst + 8192 + off) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&l01), *reinterpret_cast<uint32_t*>(&l23));
+      }
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------

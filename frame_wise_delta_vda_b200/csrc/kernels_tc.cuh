@@ -1,5 +1,5 @@
 // kernels_tc.cuh - sm_100a tensor-core kernels of the VDA path for d = 128
-// with bf16 I/O: TMA-fed tcgen05 MMAs accumulating in TMEM.
+// and d = 64 with bf16 I/O: TMA-fed tcgen05 MMAs accumulating in TMEM.
 //
 // Paper: "Video DeltaNet" (arXiv 2609.20744).
 //   k_stats_tc    Eq. 3b: A_t = K^T Diag(beta) K, B_t = V^T Diag(beta) K
@@ -7,9 +7,12 @@
 //                 on the tensor cores, written as the bf16 hi/lo operand image
 //                 the scan feeds to the tensor cores
 //   k_scan_tc     Section 2.2 + Eq. 5: S_t = (S_{t-1} + B_t) M_t, both
-//                 directions, fp32 state, 3-product bf16 hi/lo split MMAs
+//                 directions, fp32 state, 3-product bf16 hi/lo split MMAs;
+//                 per-frame chains or the chunk-wise form of Section 5
 //   k_readout_tc  Appendix A.3 (Eq. A.4) gather, Eq. 1a readout o = S~ q,
-//                 Eq. 1c RMSNorm + sigmoid gate, bf16 store
+//                 Eq. 1c RMSNorm + sigmoid gate, bf16 store (d = 128, 64)
+//   k_stats64_tc, k_scan64_tc  the d = 64 Gram kernel and scans (the inverse
+//                 at d = 64 is the FP32 Gauss-Jordan kernel of kernels_simt.cuh)
 #pragma once
 
 #include <cuda.h>
@@ -342,6 +345,232 @@ k_stats_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUte
     tmem_dealloc(tmem, 512);
   }
   if (warp == C::WARP_PROD && lane == 0 && *abort_flag) {  // let issued copies land before the CTA exits
+    for (int s = 0; s < C::NST; ++s)
+      if (last_it[s] >= 0) mbar_wait_drain(BAR(FULL + s), ((uint32_t)last_it[s] / C::NST) & 1u);
+  }
+}
+
+// ===========================================================================
+// k_stats64_tc: the Gram kernel for d = 64.  With 64 channels the roles of
+// the operands swap so that the MMA keeps M = 128: tokens on the K dimension,
+//   D[128 x 64] = [K | V]^T (beta K)_hi + [K | V]^T (beta K)_lo
+// so D[0:64, :] = A and D[64:128, :] = B (rows n of B, columns j).  Both
+// operands are MN-major 64-channel TMA boxes (64 tokens x 128 B, 128-B
+// swizzle); [K | V] is two boxes 8 KB apart (the M dimension's two 64-blocks).
+// Warps: 0-3 epilogue (TMEM lane i < 64: A row i; lane 64 + n: B row n),
+// 4-7 scale (beta K -> bf16 hi + lo), 8 TMA producer, 9 MMA issuer.  Four
+// load stages (K, V: 16 KB), two scaled buffers (hi, lo: 16 KB), two
+// 64-column TMEM accumulators.  Out: A [64][64] (symmetric, stored by
+// columns), B^T [64][64] (B^T[j][n] = B[n][j], the layout the d = 64 scan
+// reads), optionally B [n][j] for the debug output.
+// ===========================================================================
+struct Stats64Cfg {
+  static constexpr int UT = 64;
+  static constexpr int NST = 4;                      // load stages
+  static constexpr int NSC = 2;                      // scaled buffers
+  static constexpr uint32_t BLK = UT * 128;          // 8192: 64 tokens x 64 channels
+  static constexpr uint32_t STAGE = 2 * BLK;         // K, V
+  static constexpr uint32_t SCBUF = 2 * BLK;         // hi, lo
+  static constexpr uint32_t OFF_SC = NST * STAGE;
+  static constexpr int NSCALE = 128;                 // 64 rows x 2 halves of the 128-B row
+  static constexpr int WARP_PROD = 4 + NSCALE / 32;
+  static constexpr int WARP_MMA = WARP_PROD + 1;
+  static constexpr int THREADS = 32 * (WARP_MMA + 1);
+  static constexpr uint32_t BAR_OFF = OFF_SC + NSC * SCBUF;
+  static constexpr int NBAR = 2 * NST + 2 * NSC + 5;
+  static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
+};
+
+__global__ void __launch_bounds__(Stats64Cfg::THREADS, 1)
+k_stats64_tc(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+             const float* __restrict__ beta, int U, int FH, float* __restrict__ A_out, float* __restrict__ Bt_out,
+             float* __restrict__ B_full) {
+  using C = Stats64Cfg;
+  constexpr int D = 64;
+  constexpr size_t DD = 64 * 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
+  const int FULL = 0, EMPTY = C::NST, SCALED = 2 * C::NST, SEMPTY = 2 * C::NST + C::NSC,
+            TFULL = 2 * C::NST + 2 * C::NSC, TEMPTY = TFULL + 2, DRAIN = TFULL + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(BAR(FULL + s), 1);
+      mbar_init(BAR(EMPTY + s), 1);
+    }
+    for (int b = 0; b < C::NSC; ++b) {
+      mbar_init(BAR(SCALED + b), C::NSCALE);
+      mbar_init(BAR(SEMPTY + b), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(BAR(TFULL + b), 1);
+      mbar_init(BAR(TEMPTY + b), 128);
+    }
+    mbar_init(BAR(DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  grid_wait_prerequisites();   // (see k_stats_tc)
+  grid_launch_dependents();
+  const uint32_t tmem = *tmem_slot;
+  const int nt = (U + C::UT - 1) / C::UT;
+  int last_it[C::NST];
+  for (int s = 0; s < C::NST; ++s) last_it[s] = -1;
+
+  if (warp == C::WARP_PROD) {
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int fh = blockIdx.x; ok && fh < FH; fh += gridDim.x) {
+        for (int tile = 0; tile < nt; ++tile, ++it) {
+          const uint32_t s = it % C::NST, ph = (it / C::NST) & 1u;
+          if (!mbar_wait(BAR(EMPTY + s), ph ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(BAR(FULL + s), 2 * C::BLK);
+          const uint32_t st = sbase + s * C::STAGE;
+          tma_load_3d(st, &tmK, 0, tile * C::UT, fh, BAR(FULL + s));
+          tma_load_3d(st + C::BLK, &tmV, 0, tile * C::UT, fh, BAR(FULL + s));
+          last_it[s] = (int)it;
+        }
+      }
+    }
+  } else if (warp == C::WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t kId = idesc_bf16(128, 64, 1, 1);   // A = [K | V], B = beta K, both MN-major
+      uint32_t it = 0, lf = 0;
+      bool ok = true;
+      for (int fh = blockIdx.x; ok && fh < FH; fh += gridDim.x, ++lf) {
+        const uint32_t buf = lf & 1u, bph = (lf >> 1) & 1u;
+        if (!mbar_wait(BAR(TEMPTY + buf), bph ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * 64u;
+        for (int tile = 0; tile < nt; ++tile, ++it) {
+          const uint32_t s = it % C::NST;
+          const uint32_t b = it % C::NSC, bph2 = (it / C::NSC) & 1u;
+          if (!mbar_wait(BAR(SCALED + b), bph2, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t st = sbase + s * C::STAGE;
+          const uint32_t sc = sbase + C::OFF_SC + b * C::SCBUF;
+#pragma unroll
+          for (int ks = 0; ks < C::UT / 16; ++ks) {
+            const uint32_t ko = (uint32_t)ks * 2048u;
+            const uint64_t a = desc_sw128(st + ko, C::BLK, 1024);
+            mma_bf16_ss(d, a, desc_sw128(sc + ko, C::BLK, 1024), kId, (tile | ks) != 0);
+            mma_bf16_ss(d, a, desc_sw128(sc + C::BLK + ko, C::BLK, 1024), kId, 1u);
+          }
+          mma_commit(BAR(EMPTY + s));
+          mma_commit(BAR(SEMPTY + b));
+        }
+        if (!ok) break;
+        mma_commit(BAR(TFULL + buf));
+      }
+      mma_commit(BAR(DRAIN));
+      mbar_wait_drain(BAR(DRAIN), 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------- beta * K -> bf16 hi + lo in the same swizzled position:
+    // thread = (token row r, half qt of the row's eight 16-B chunks)
+    const int st_id = tid - 128;
+    const int r = st_id & 63, qt = st_id >> 6;
+    auto beta_at = [&](int f, int tl) -> float {
+      const int u = tl * C::UT + r;
+      return (f < FH && u < U) ? __ldg(beta + (size_t)f * U + u) : 0.f;
+    };
+    uint32_t it = 0;
+    int fh = blockIdx.x, tile = 0;
+    float b_next = beta_at(fh, 0);
+    while (fh < FH) {
+      const float b = b_next;
+      int nfh = fh, ntile = tile + 1;
+      if (ntile == nt) { ntile = 0; nfh += gridDim.x; }
+      b_next = beta_at(nfh, ntile);
+      const uint32_t s = it % C::NST, ph = (it / C::NST) & 1u;
+      const uint32_t sb = it % C::NSC, sph = (it / C::NSC) & 1u;
+      if (!mbar_wait(BAR(FULL + s), ph, abort_flag)) break;
+      if (!mbar_wait(BAR(SEMPTY + sb), sph ^ 1u, abort_flag)) break;
+      const uint32_t ksrc = sbase + s * C::STAGE + (uint32_t)r * 128u;
+      const uint32_t hdst = sbase + C::OFF_SC + sb * C::SCBUF + (uint32_t)r * 128u;
+      const uint32_t ldst = hdst + C::BLK;
+      uint32_t pos[4];
+      uint4 kvs[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        pos[c] = (uint32_t)((4 * qt + c + r) & 7) * 16u;   // rotated across rows: conflict-free
+        kvs[c] = ld_shared_v4(ksrc + pos[c]);
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t w[4] = {kvs[c].x, kvs[c].y, kvs[c].z, kvs[c].w};
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float x0 = __uint_as_float(w[q] << 16) * b;
+          const float x1 = __uint_as_float(w[q] & 0xFFFF0000u) * b;
+          hw[q] = pack_bf16(x0, x1);
+          const float h0 = __uint_as_float(hw[q] << 16), h1 = __uint_as_float(hw[q] & 0xFFFF0000u);
+          lw[q] = pack_bf16(x0 - h0, x1 - h1);
+        }
+        st_shared_v4(hdst + pos[c], make_uint4(hw[0], hw[1], hw[2], hw[3]));
+        st_shared_v4(ldst + pos[c], make_uint4(lw[0], lw[1], lw[2], lw[3]));
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(SCALED + sb));
+      ++it;
+      fh = nfh;
+      tile = ntile;
+    }
+  } else {
+    // ---------------- epilogue: TMEM lane i; i < 64: A row i, stored as A[c][i]
+    // (A is symmetric; 32 lanes store 128 contiguous bytes); i = 64 + n: B row
+    // n, stored as B^T[j][n]
+    const int i = warp * 32 + lane;
+    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    uint32_t lf = 0;
+    for (int fh = blockIdx.x; fh < FH; fh += gridDim.x, ++lf) {
+      const uint32_t buf = lf & 1u, bph = (lf >> 1) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(TFULL + buf), bph, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t tA = tmem + buf * 64u;
+      uint32_t v0[32], v1[32];
+      tmem_ld32(lb + tA, v0);
+      tmem_ld32(lb + tA + 32u, v1);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(BAR(TEMPTY + buf));
+      float* dst = (i < D ? A_out : Bt_out) + (size_t)fh * DD + (i & 63);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) dst[(size_t)c * D] = __uint_as_float(v0[c]);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) dst[(size_t)(32 + c) * D] = __uint_as_float(v1[c]);
+      if (B_full && i >= D) {   // debug output: B[n][j]
+        float* bf = B_full + (size_t)fh * DD + (size_t)(i - D) * D;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) bf[c] = __uint_as_float(v0[c]);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) bf[32 + c] = __uint_as_float(v1[c]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+  if (warp == C::WARP_PROD && lane == 0 && *abort_flag) {
     for (int s = 0; s < C::NST; ++s)
       if (last_it[s] >= 0) mbar_wait_drain(BAR(FULL + s), ((uint32_t)last_it[s] / C::NST) & 1u);
   }
@@ -1146,6 +1375,220 @@ __global__ void __launch_bounds__(ScanCfg::THREADS, 1) k_scan_tc(const ScanArgs 
 }
 
 // ===========================================================================
+// k_scan64_tc: the scans for d = 64.  One CTA runs both chains of a (b, h):
+// chain 0 forward, chain 1 reverse, in lockstep.  A 64 x 64 update would
+// give the MMA M = 64, so the two chains share one M = 128, N = 128 MMA:
+//   D[j'][n'] = sum_k A[j'][k] X[n'][k],   A = [M_fwd^T ; M_rev^T] (j' = 64 c + j),
+//                                          X = [X_fwd ; X_rev]     (n' = 64 c + n)
+// of which the diagonal blocks D[64c + j][64c + n] = (X_c M_c)[n][j] are the
+// two chains' new states (the off-diagonal blocks are not read).  Operands
+// are bf16 hi / lo (3 products), k = 0..63 in four steps of 16.
+// Warps 0-3: state (warp w: chain w / 2, thread j = (w & 1) * 32 + lane owns
+// column j of its chain's S = TMEM lane 64 c + j); warp 4: bulk copies of
+// the two chains' M images (two stages); warp 5: MMA issuer.
+// Operand images (d = 64): 64 rows of 128 B, 128-B swizzle, 8 KB each; M
+// image element (j, k) = M[k][j] in row k; X image element (n, k) in row k.
+// In: M images [BH][T] (hi 8 KB, lo 8 KB), B^T [BH][T][64][64].
+// Out: boundary states [2][BH][NC + 1][64][64] as for d = 128.
+// ===========================================================================
+struct Scan64Cfg {
+  static constexpr int THREADS = 192;
+  static constexpr int PREFETCH = 3;
+  static constexpr int WARP_PROD = 4;
+  static constexpr int WARP_MMA = 5;
+  static constexpr uint32_t IMG = 8192;                 // one 64 x 64 bf16 image
+  static constexpr uint32_t MST = 4 * IMG;              // stage: hi c0, hi c1, lo c0, lo c1
+  static constexpr uint32_t OFF_M = 0;                  // 2 stages
+  static constexpr uint32_t OFF_X = 2 * MST;            // hi c0, hi c1, lo c0, lo c1
+  static constexpr uint32_t BAR_OFF = OFF_X + 4 * IMG;
+  static constexpr int NBAR = 2 + 2 + 1 + 1 + 1;         // mfull[2], mempty[2], xfull, dfull, drain
+  static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
+};
+constexpr uint32_t kImg64Bytes = 2 * Scan64Cfg::IMG;    // hi + lo image of one 64 x 64 matrix
+
+__global__ void __launch_bounds__(Scan64Cfg::THREADS, 1)
+k_scan64_tc(const uint8_t* __restrict__ Mimg, const float* __restrict__ Bt, const float* __restrict__ S0f,
+            const float* __restrict__ S0r, const float* __restrict__ alpha, float* __restrict__ states, int BH,
+            int T, int chunk, int NC) {
+  using C = Scan64Cfg;
+  constexpr int D = 64;
+  constexpr size_t DD = 64 * 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8u * (uint32_t)i; };
+  const int MFULL = 0, MEMPTY = 2, XFULL = 4, DFULL = 5, DRAIN = 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::BAR_OFF + C::NBAR * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;
+  auto frame_of = [&](int c, int i) { return c == 0 ? i : T - 1 - i; };
+  if (tid == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(MFULL + s), 1);
+      mbar_init(BAR(MEMPTY + s), 1);
+    }
+    mbar_init(BAR(XFULL), 128);
+    mbar_init(BAR(DFULL), 1);
+    mbar_init(BAR(DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::WARP_MMA) {
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  grid_wait_prerequisites();   // the M images and B^T are complete
+  grid_launch_dependents();
+  const uint32_t tmem = *tmem_slot;
+  int last_i[2] = {-1, -1};
+
+  if (warp == C::WARP_PROD) {
+    if (lane == 0) {
+      for (int i = 0; i < T; ++i) {
+        const uint32_t s = (uint32_t)i & 1u, ph = ((uint32_t)i >> 1) & 1u;
+        if (!mbar_wait(BAR(MEMPTY + s), ph ^ 1u, abort_flag)) break;
+        mbar_arrive_expect_tx(BAR(MFULL + s), 4 * C::IMG);
+        const uint32_t dst = sbase + C::OFF_M + s * C::MST;
+        for (int c = 0; c < 2; ++c) {
+          const uint8_t* src = Mimg + ((size_t)bh * T + frame_of(c, i)) * kImg64Bytes;
+          bulk_load(dst + (uint32_t)c * C::IMG, src, C::IMG, BAR(MFULL + s));                 // hi
+          bulk_load(dst + 2u * C::IMG + (uint32_t)c * C::IMG, src + C::IMG, C::IMG, BAR(MFULL + s));  // lo
+          if (i + C::PREFETCH < T) {
+            const size_t fa = (size_t)bh * T + frame_of(c, i + C::PREFETCH);
+            bulk_prefetch_l2(Mimg + fa * kImg64Bytes, kImg64Bytes);
+            bulk_prefetch_l2(Bt + fa * DD, (uint32_t)(DD * sizeof(float)));
+          }
+        }
+        last_i[s] = i;
+      }
+    }
+  } else if (warp == C::WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t kId = idesc_bf16(128, 128, 1, 1);   // both MN-major
+      for (int i = 0; i < T; ++i) {
+        const uint32_t s = (uint32_t)i & 1u, ph = ((uint32_t)i >> 1) & 1u;
+        if (!mbar_wait(BAR(MFULL + s), ph, abort_flag)) break;
+        if (!mbar_wait(BAR(XFULL), (uint32_t)i & 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t mh = sbase + C::OFF_M + s * C::MST, ml = mh + 2u * C::IMG;
+        const uint32_t xh = sbase + C::OFF_X, xl = xh + 2u * C::IMG;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t ko = (uint32_t)ks * 2048u;   // 16 k-rows
+          const uint64_t a_h = desc_sw128(mh + ko, C::IMG, 1024), a_l = desc_sw128(ml + ko, C::IMG, 1024);
+          const uint64_t b_h = desc_sw128(xh + ko, C::IMG, 1024), b_l = desc_sw128(xl + ko, C::IMG, 1024);
+          mma_bf16_ss(tmem, a_h, b_h, kId, ks != 0);
+          mma_bf16_ss(tmem, a_h, b_l, kId, 1u);
+          mma_bf16_ss(tmem, a_l, b_h, kId, 1u);
+        }
+        mma_commit(BAR(DFULL));
+        mma_commit(BAR(MEMPTY + s));
+      }
+      mma_commit(BAR(DRAIN));
+      mbar_wait_drain(BAR(DRAIN), 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- state warps
+    const int c = warp >> 1;                 // chain: 0 forward, 1 reverse
+    const int j = (warp & 1) * 32 + lane;    // column j of the chain's S
+    const float* S0 = c == 0 ? S0f : S0r;
+    float* st = states + ((size_t)c * BH + bh) * (size_t)(NC + 1) * DD;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16) + 64u * (uint32_t)c;
+    const uint32_t xrow = sbase + C::OFF_X + (uint32_t)c * C::IMG + (uint32_t)j * 128u;
+    const uint32_t jsw = (uint32_t)(j & 7);
+    float bnext[64];
+    auto load_b = [&](int fr) {   // B[n][j] = B^T[j][n], n = 0..63: one contiguous row
+      const float4* src = reinterpret_cast<const float4*>(Bt + ((size_t)bh * T + fr) * DD + (size_t)j * D);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const float4 v = __ldg(src + q);
+        bnext[4 * q] = v.x; bnext[4 * q + 1] = v.y; bnext[4 * q + 2] = v.z; bnext[4 * q + 3] = v.w;
+      }
+    };
+    {   // initial state: the first boundary, X_0 = S0 Diag(alpha) + B
+      const int j0 = c == 0 ? 0 : NC;
+      const int f0 = frame_of(c, 0);
+      load_b(f0);
+      const float a0 = alpha ? __ldg(alpha + ((size_t)bh * T + f0) * D + j) : 1.f;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int n = 8 * cc + e;
+          const float s0 = S0 ? __ldg(S0 + (size_t)bh * DD + (size_t)n * D + j) : 0.f;
+          st[(size_t)j0 * DD + (size_t)n * D + j] = s0;
+          x[e] = fmaf(s0, a0, bnext[n]);
+        }
+        const uint32_t o = xrow + (((uint32_t)cc ^ jsw) << 4);
+        st_chunk_hilo(o, o + 2u * C::IMG, x);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(XFULL));
+    }
+    for (int i = 0; i < T; ++i) {
+      const bool more = i + 1 < T;
+      const int t = frame_of(c, i);
+      int jb = -1;
+      if (c == 0) {
+        if ((t + 1) % chunk == 0 || t == T - 1) jb = (t + chunk) / chunk;
+      } else if (t % chunk == 0) {
+        jb = t / chunk;
+      }
+      float anext = 1.f;
+      if (more) {
+        load_b(frame_of(c, i + 1));
+        if (alpha) anext = __ldg(alpha + ((size_t)bh * T + frame_of(c, i + 1)) * D + j);
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(BAR(DFULL), (uint32_t)i & 1u, abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        uint32_t v[16];
+        tmem_ld16(trow + cb * 16, v);
+        tmem_wait_ld();
+        if (jb >= 0) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) st[(size_t)jb * DD + (size_t)(cb * 16 + e) * D + j] = __uint_as_float(v[e]);
+        }
+        if (more) {
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) {
+            float x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = fmaf(__uint_as_float(v[8 * q2 + e]), anext, bnext[cb * 16 + 8 * q2 + e]);
+            const uint32_t c8 = (uint32_t)(2 * cb + q2);
+            const uint32_t o = xrow + ((c8 ^ jsw) << 4);
+            st_chunk_hilo(o, o + 2u * C::IMG, x);
+          }
+        }
+      }
+      if (more) {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(BAR(XFULL));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+  if (warp == C::WARP_PROD && lane == 0 && *abort_flag) {
+    for (int s = 0; s < 2; ++s)
+      if (last_i[s] >= 0) mbar_wait_drain(BAR(MFULL + s), ((uint32_t)last_i[s] >> 1) & 1u);
+  }
+}
+
+// ===========================================================================
 // k_readout_tc: out = sigmoid(g) * w * o / sqrt(mean(o^2) + eps), o = S~ q.
 // Work = 128-token tiles of each (b, h, chunk)'s contiguous token range; a
 // persistent CTA takes a contiguous run of tiles.  Per tile the MMA computes
@@ -1165,22 +1608,28 @@ __global__ void __launch_bounds__(ScanCfg::THREADS, 1) k_scan_tc(const ScanArgs 
 // warp 10: gate producer (separate producers keep Q loads running ahead of
 // the epilogue's release of gate stages).
 // ===========================================================================
-struct ReadoutCfg {
+template <int D>   // d_k = d_v = 128 or 64
+struct ReadoutCfgT {
   static constexpr int NEPI = 256;                             // epilogue threads (warps 0-7)
   static constexpr int WARP_Q = 8, WARP_MMA = 9, WARP_G = 10;
   static constexpr int THREADS = 352;
   static constexpr int TILE = 128;
-  static constexpr uint32_t TILE_BYTES = TILE * 256;           // 128 rows x 128 bf16
-  static constexpr uint32_t OFF_S = 0;                         // S~ hi (32 KB) + lo (32 KB)
-  static constexpr uint32_t OFF_Q = kImgBytes;                 // 2 x 32 KB
+  static constexpr int NB = D / 64;                            // 64-channel boxes of a tile
+  static constexpr int HALF = D / 2;                           // output columns per epilogue thread
+  static constexpr uint32_t BOX_BYTES = TILE * 128;            // 128 rows x 64 bf16
+  static constexpr uint32_t TILE_BYTES = NB * BOX_BYTES;       // 128 rows x D bf16
+  static constexpr uint32_t SIMG = D * D * 2;                  // one bf16 S~ image (hi or lo)
+  static constexpr uint32_t OFF_S = 0;                         // S~ hi + lo
+  static constexpr uint32_t OFF_Q = 2 * SIMG;                  // 2 Q stages
   static constexpr int NG = 2;                                  // gate stages (also hold the output)
-  static constexpr uint32_t OFF_G = kImgBytes + 2 * TILE_BYTES; // NG x 32 KB
-  static constexpr uint32_t OFF_W = OFF_G + NG * TILE_BYTES;    // 128 floats
+  static constexpr uint32_t OFF_G = OFF_Q + 2 * TILE_BYTES;     // NG gate stages
+  static constexpr uint32_t OFF_W = OFF_G + NG * TILE_BYTES;    // D floats
   static constexpr uint32_t BAR_OFF = OFF_W + 512;
   // qfull[2], qempty[2], gfull[NG], gout[NG], tfull[2], tempty[2], sready, drain
   static constexpr int NBAR = 10 + 2 * NG;
   static constexpr size_t SMEM = BAR_OFF + NBAR * 8 + 16 + 1024;
 };
+using ReadoutCfg = ReadoutCfgT<128>;
 
 struct ReadoutGeom {
   int BH, T, U, chunk, NC, window;
@@ -1205,12 +1654,14 @@ __device__ __forceinline__ void tile_coords(const ReadoutGeom& g, long long gt, 
   rows = (f1 - f0) * g.U;
 }
 
-__global__ void __launch_bounds__(ReadoutCfg::THREADS, 1)
+template <int D>
+__global__ void __launch_bounds__(ReadoutCfgT<D>::THREADS, 1)
 k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmG,
              const __grid_constant__ CUtensorMap tmO,
              const float* __restrict__ w, const float* __restrict__ states, const float* __restrict__ bridge,
              __nv_bfloat16* __restrict__ out, ReadoutGeom g, float eps) {
-  using C = ReadoutCfg;
+  using C = ReadoutCfgT<D>;
+  constexpr size_t DD = (size_t)D * D;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sbase = smem_u32(smem);
@@ -1243,14 +1694,14 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     fence_mbar_init();
   }
   if (warp == C::WARP_MMA) {
-    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_alloc(smem_u32(tmem_slot), 2 * D);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   grid_wait_prerequisites();   // boundary states are complete (see k_stats_tc)
   grid_launch_dependents();
-  if (tid < kD) sw[tid] = 0.5f * w[tid];
+  if (tid < D) sw[tid] = 0.5f * w[tid];
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -1274,13 +1725,13 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         const uint32_t src = base + s * C::TILE_BYTES;
         if (g.frame_out) {   // rows past the frame's U are outside the map: not written
           const int fh = bh * g.T + c;
-          tma_store_3d(&tmO, src, 0, tr, fh);
-          tma_store_3d(&tmO, src + C::TILE_BYTES / 2, 64, tr, fh);
+#pragma unroll
+          for (int bx = 0; bx < C::NB; ++bx) tma_store_3d(&tmO, src + bx * C::BOX_BYTES, 64 * bx, tr, fh);
           bulk_commit_group();
         } else if (tr + C::TILE <= rows) {
           const int row0 = (int)((long long)bh * tokens_per_head + (long long)c * g.unit * g.U + tr);
-          tma_store_2d(&tmO, src, 0, row0);
-          tma_store_2d(&tmO, src + C::TILE_BYTES / 2, 64, row0);
+#pragma unroll
+          for (int bx = 0; bx < C::NB; ++bx) tma_store_2d(&tmO, src + bx * C::BOX_BYTES, 64 * bx, row0);
           bulk_commit_group();
         }
       };
@@ -1301,8 +1752,8 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         const int FULLB = is_q ? QFULL : GFULL;
         mbar_arrive_expect_tx(BAR(FULLB + s), C::TILE_BYTES);
         const uint32_t dst = base + s * C::TILE_BYTES;
-        tma_load_2d(dst, map, 0, row0, BAR(FULLB + s));
-        tma_load_2d(dst + C::TILE_BYTES / 2, map, 64, row0, BAR(FULLB + s));
+#pragma unroll
+        for (int bx = 0; bx < C::NB; ++bx) tma_load_2d(dst + bx * C::BOX_BYTES, map, 64 * bx, row0, BAR(FULLB + s));
         last[s] = k;
       }
       if (!is_q && ok) {   // the last NG output tiles
@@ -1318,8 +1769,8 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
   } else if (warp == C::WARP_MMA) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kId = idesc_bf16(128, 128, 0, 0);   // both K-major
-      const uint32_t sh = sbase + C::OFF_S, sl = sh + kImgHalf;
+      constexpr uint32_t kId = idesc_bf16(128, D, 0, 0);   // both K-major
+      const uint32_t sh = sbase + C::OFF_S, sl = sh + C::SIMG;
       int k = 0, npair = 0, prev_bh = -1, prev_c = -1;
       for (long long gt = t_begin; gt < t_end; ++gt, ++k) {
         int bh, c, tr, rows;
@@ -1335,13 +1786,15 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         if (!mbar_wait(BAR(TEMPTY + s), ph ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t q = sbase + C::OFF_Q + s * C::TILE_BYTES;
-        const uint32_t d = tmem + s * 128u;
+        const uint32_t d = tmem + s * (uint32_t)D;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t o = (uint32_t)(ks >> 2) * 16384u + (uint32_t)(ks & 3) * 32u;
-          const uint64_t a = desc_sw128(q + o, 16, 1024);
-          mma_bf16_ss(d, a, desc_sw128(sh + o, 16, 1024), kId, ks != 0);
-          mma_bf16_ss(d, a, desc_sw128(sl + o, 16, 1024), kId, 1u);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          // k-block ks / 4 of 64 channels: a 16 KB box of Q, a (D x 128 B) block of S~
+          const uint32_t kc = (uint32_t)(ks & 3) * 32u;
+          const uint64_t a = desc_sw128(q + (uint32_t)(ks >> 2) * C::BOX_BYTES + kc, 16, 1024);
+          const uint32_t so = (uint32_t)(ks >> 2) * (uint32_t)(D * 128) + kc;
+          mma_bf16_ss(d, a, desc_sw128(sh + so, 16, 1024), kId, ks != 0);
+          mma_bf16_ss(d, a, desc_sw128(sl + so, 16, 1024), kId, 1u);
         }
         mma_commit(BAR(QEMPTY + s));
         mma_commit(BAR(TFULL + s));
@@ -1355,25 +1808,27 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     const int r = (warp & 3) * 32 + lane, ch = warp >> 2;
     const uint32_t trow_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t simg_s = sbase + C::OFF_S;
-    const uint32_t sw_s = sbase + C::OFF_W + 256u * (uint32_t)ch;   // w/2 of this half
+    const uint32_t sw_s = sbase + C::OFF_W + (uint32_t)(C::HALF * 4) * (uint32_t)ch;   // w/2 of this half
     int k = 0, prev_bh = -1, prev_c = -1;
-    const size_t sdir = (size_t)g.BH * (size_t)(g.NC + 1) * kDD;
+    const size_t sdir = (size_t)g.BH * (size_t)(g.NC + 1) * DD;
     for (long long gt = t_begin; gt < t_end; ++gt, ++k) {
       int bh, c, tr, rows;
       tile_coords(g, gt, bh, c, tr, rows);
       if (bh != prev_bh || c != prev_c) {
         // build S~ = fwd[max(0, c-w)] + rev[min(NC, c+w+1)] (chunk c of this unit),
         // with the decay bridge fwd Diag(bl) + rev Diag(br) of frame u (Eq. A.4):
-        // row i = r, this half's columns
+        // row i = r (rows below D), this half's columns
         const int cc_ = (c * g.unit) / g.chunk;
         const int jf = max(0, cc_ - g.window), jr = min(g.NC, cc_ + g.window + 1);
-        const float* bl = bridge ? bridge + (((size_t)bh * g.T + c) * 2) * kD + 64 * ch : nullptr;
+        const int rs = r < D ? r : 0;
+        const float* bl = bridge ? bridge + (((size_t)bh * g.T + c) * 2) * D + C::HALF * ch : nullptr;
         const float* Sf =
-            states + (size_t)bh * (size_t)(g.NC + 1) * kDD + (size_t)jf * kDD + (size_t)r * kD + 64 * ch;
-        const float* Sr = states + sdir + (size_t)bh * (size_t)(g.NC + 1) * kDD + (size_t)jr * kD * kD +
-                          (size_t)r * kD + 64 * ch;
+            states + (size_t)bh * (size_t)(g.NC + 1) * DD + (size_t)jf * DD + (size_t)rs * D + C::HALF * ch;
+        const float* Sr = states + sdir + (size_t)bh * (size_t)(g.NC + 1) * DD + (size_t)jr * DD +
+                          (size_t)rs * D + C::HALF * ch;
 #pragma unroll 4
-        for (int cc = 0; cc < 8; ++cc) {
+        for (int cc = 0; cc < C::HALF / 8; ++cc) {
+          if (r >= D) break;
           const float4 f0 = __ldg(reinterpret_cast<const float4*>(Sf + cc * 8));
           const float4 f1 = __ldg(reinterpret_cast<const float4*>(Sf + cc * 8 + 4));
           const float4 r0v = __ldg(reinterpret_cast<const float4*>(Sr + cc * 8));
@@ -1383,8 +1838,8 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
           if (bl) {
             const float4 a0 = __ldg(reinterpret_cast<const float4*>(bl + cc * 8));
             const float4 a1 = __ldg(reinterpret_cast<const float4*>(bl + cc * 8 + 4));
-            const float4 b0 = __ldg(reinterpret_cast<const float4*>(bl + kD + cc * 8));
-            const float4 b1 = __ldg(reinterpret_cast<const float4*>(bl + kD + cc * 8 + 4));
+            const float4 b0 = __ldg(reinterpret_cast<const float4*>(bl + D + cc * 8));
+            const float4 b1 = __ldg(reinterpret_cast<const float4*>(bl + D + cc * 8 + 4));
             x[0] = fmaf(f0.x, a0.x, r0v.x * b0.x); x[1] = fmaf(f0.y, a0.y, r0v.y * b0.y);
             x[2] = fmaf(f0.z, a0.z, r0v.z * b0.z); x[3] = fmaf(f0.w, a0.w, r0v.w * b0.w);
             x[4] = fmaf(f1.x, a1.x, r1v.x * b1.x); x[5] = fmaf(f1.y, a1.y, r1v.y * b1.y);
@@ -1399,9 +1854,11 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             hw[q] = pack_bf16(h0, h1);
             lw[q] = pack_bf16(l0, l1);
           }
-          const uint32_t off = ximg_offset(r, 64 * ch + cc * 8);   // row i = r, columns k
+          // row i = r, columns k: k-block k / 64 of D rows x 128 B, 128-B swizzle
+          const uint32_t kk = (uint32_t)(C::HALF * ch + cc * 8);
+          const uint32_t off = (kk >> 6) * (uint32_t)(D * 128) + sw128_offset((uint32_t)r, kk & 63u);
           st_shared_v4(simg_s + off, make_uint4(hw[0], hw[1], hw[2], hw[3]));
-          st_shared_v4(simg_s + kImgHalf + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+          st_shared_v4(simg_s + C::SIMG + off, make_uint4(lw[0], lw[1], lw[2], lw[3]));
         }
         fence_proxy_async_smem();
         mbar_arrive(BAR(SREADY));
@@ -1412,54 +1869,49 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(TFULL + s), ph, abort_flag))) break;
       tc_fence_after();
       // sum of squares over the whole row (both halves, fixed order); keep this half
-      float o[64];
+      float o[C::HALF];
       float ss = 0.f;
-      const uint32_t trow = trow_base + s * 128u;
+      const uint32_t trow = trow_base + s * (uint32_t)D;
 #pragma unroll
       for (int j2 = 0; j2 < 2; ++j2) {
-        uint32_t v0[32], v1[32];
-        tmem_ld32(trow + 64u * j2, v0);
-        tmem_ld32(trow + 64u * j2 + 32u, v1);
-        tmem_wait_ld();
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          const float a0 = __uint_as_float(v0[c2]);
-          ss = fmaf(a0, a0, ss);
-        }
-#pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          const float a1 = __uint_as_float(v1[c2]);
-          ss = fmaf(a1, a1, ss);
-        }
-        if (j2 == ch) {
+        for (int j3 = 0; j3 < C::HALF / 32; ++j3) {
+          uint32_t v0[32];
+          tmem_ld32(trow + (uint32_t)(C::HALF * j2 + 32 * j3), v0);
+          tmem_wait_ld();
 #pragma unroll
           for (int c2 = 0; c2 < 32; ++c2) {
-            o[c2] = __uint_as_float(v0[c2]);
-            o[32 + c2] = __uint_as_float(v1[c2]);
+            const float a0 = __uint_as_float(v0[c2]);
+            ss = fmaf(a0, a0, ss);
+          }
+          if (j2 == ch) {
+#pragma unroll
+            for (int c2 = 0; c2 < 32; ++c2) o[32 * j3 + c2] = __uint_as_float(v0[c2]);
           }
         }
       }
       tc_fence_before();
       mbar_arrive(BAR(TEMPTY + s));
-      const float rinv = rsqrtf(ss * (1.0f / kD) + eps);
+      const float rinv = rsqrtf(ss * (1.0f / D) + eps);
       const uint32_t sg = (uint32_t)(k % C::NG), phg = (uint32_t)(k / C::NG) & 1u;
       if (!__all_sync(0xffffffffu, mbar_wait(BAR(GFULL + sg), phg, abort_flag))) break;
-      const uint32_t gt_s = sbase + C::OFF_G + sg * C::TILE_BYTES + (uint32_t)ch * (C::TILE_BYTES / 2);
+      const uint32_t gt_s = sbase + C::OFF_G + sg * C::TILE_BYTES;
       const bool valid = tr + r < rows;
       // a tile inside its chunk leaves by TMA from the gate stage (y replaces
       // g in place); the chunk's last, partial tile by per-row stores
       const bool tma_out = g.frame_out || tr + C::TILE <= rows;
       __nv_bfloat16* orow =
-          out + ((size_t)bh * tokens_per_head + (size_t)c * g.unit * g.U + tr + r) * kD + 64 * ch;
+          out + ((size_t)bh * tokens_per_head + (size_t)c * g.unit * g.U + tr + r) * D + C::HALF * ch;
 #pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {   // 4 chunks of 8 columns at a time, loads first
+      for (int cb = 0; cb < C::HALF / 32; ++cb) {   // 4 chunks of 8 columns at a time, loads first
         uint4 gv[4];
         float4 wv[8];
         uint32_t off[4];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const int cc = 4 * cb + q4;
-          off[q4] = sw128_offset((uint32_t)r, (uint32_t)(cc * 8));
+          const uint32_t col = (uint32_t)(C::HALF * ch + cc * 8);   // column of the tile: box col / 64
+          off[q4] = (col >> 6) * C::BOX_BYTES + sw128_offset((uint32_t)r, col & 63u);
           gv[q4] = ld_shared_v4(gt_s + off[q4]);
           wv[2 * q4] = ld_shared_f4(sw_s + (uint32_t)cc * 32u);
           wv[2 * q4 + 1] = ld_shared_f4(sw_s + (uint32_t)cc * 32u + 16u);
@@ -1494,7 +1946,7 @@ k_readout_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
   __syncthreads();
   if (warp == C::WARP_MMA) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 2 * D);
   }
   if ((warp == C::WARP_Q || warp == C::WARP_G) && lane == 0 && *abort_flag) {  // let issued copies land
     const int* last = warp == C::WARP_Q ? last_q : last_g;
@@ -1561,11 +2013,13 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // bf16 tensor [outer][mid][128] with a box of 64 x box_mid x 1, 128-B swizzle
-inline bool encode_bf16_3d(CUtensorMap* m, const void* base, uint64_t mid, uint64_t outer, uint32_t box_mid) {
+// bf16 tensors with `width` (64 or 128) channels per row, 64-channel boxes
+inline bool encode_bf16_3d(CUtensorMap* m, const void* base, uint64_t mid, uint64_t outer, uint32_t box_mid,
+                           uint32_t width = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {128, mid, outer};
-  cuuint64_t strides[2] = {256, mid * 256};
+  cuuint64_t dims[3] = {width, mid, outer};
+  cuuint64_t strides[2] = {2ull * width, mid * 2ull * width};
   cuuint32_t box[3] = {64, box_mid, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
@@ -1574,11 +2028,12 @@ inline bool encode_bf16_3d(CUtensorMap* m, const void* base, uint64_t mid, uint6
 }
 
 // bf16 matrix [rows][128] with a box of 64 x box_rows, 128-B swizzle
-inline bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+inline bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows,
+                           uint32_t width = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {128, rows};
-  cuuint64_t strides[1] = {256};
+  cuuint64_t dims[2] = {width, rows};
+  cuuint64_t strides[1] = {2ull * width};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
@@ -1691,6 +2146,7 @@ inline int launch_scan_chunked(const uint8_t* Mimg, const float* Bm, const float
   return launch_scan_mode<kScanChunks>(chains, dim3((unsigned)BH, 2u), s);
 }
 
+template <int D>
 inline int launch_readout(const void* Q, const void* G, const float* w, const float* states, const float* bridge,
                           void* out, size_t BH, int T, int U, int chunk, int NC, int window, float eps,
                           cudaStream_t s) {
@@ -1709,15 +2165,16 @@ inline int launch_readout(const void* Q, const void* G, const float* w, const fl
   g.total = (long long)BH * g.tph;
   const uint64_t rows = (uint64_t)BH * T * U;
   CUtensorMap tmQ, tmG, tmO;
-  const bool okO = g.frame_out ? encode_bf16_3d(&tmO, out, (uint64_t)U, (uint64_t)BH * T, ReadoutCfg::TILE)
-                               : encode_bf16_2d(&tmO, out, rows, ReadoutCfg::TILE);
-  if (!encode_bf16_2d(&tmQ, Q, rows, ReadoutCfg::TILE) || !encode_bf16_2d(&tmG, G, rows, ReadoutCfg::TILE) || !okO)
+  using RC = ReadoutCfgT<D>;
+  const bool okO = g.frame_out ? encode_bf16_3d(&tmO, out, (uint64_t)U, (uint64_t)BH * T, RC::TILE, D)
+                               : encode_bf16_2d(&tmO, out, rows, RC::TILE, D);
+  if (!encode_bf16_2d(&tmQ, Q, rows, RC::TILE, D) || !encode_bf16_2d(&tmG, G, rows, RC::TILE, D) || !okO)
     return VDA_ERR_CUDA;
-  if (cudaFuncSetAttribute(k_readout_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ReadoutCfg::SMEM) !=
+  if (cudaFuncSetAttribute(k_readout_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RC::SMEM) !=
       cudaSuccess)
     return VDA_ERR_CUDA;
   const int grid = (int)std::min<long long>(g.total, (long long)num_sms());
-  return launch_pdl("k_readout_tc", k_readout_tc, dim3(grid), dim3(ReadoutCfg::THREADS), ReadoutCfg::SMEM, s, tmQ,
+  return launch_pdl("k_readout_tc", k_readout_tc<D>, dim3(grid), dim3(RC::THREADS), RC::SMEM, s, tmQ,
                     tmG, tmO, w, states, bridge, static_cast<__nv_bfloat16*>(out), g, eps);
 }
 
@@ -1725,13 +2182,13 @@ inline int launch_readout(const void* Q, const void* G, const float* w, const fl
 
 // ---------------------------------------------------------------------------
 // path selection and the staged launch used by vda.cu
-inline bool tc_path_supported(int d, int dtype) { return d == 128 && dtype == VDA_BF16; }
+inline bool tc_path_supported(int d, int dtype) { return (d == 128 || d == 64) && dtype == VDA_BF16; }
 
 // extra workspace of the tensor-core path: the M hi/lo operand images
 // (64 KB per frame-head), next to A
 inline size_t tc_extra_workspace_bytes(bool tc, size_t FH, int d) {
-  (void)d;
-  return tc ? FH * (size_t)tc::kImgBytes : 0;
+  if (!tc) return 0;
+  return FH * (size_t)(d == 64 ? tc::kImg64Bytes : tc::kImgBytes);
 }
 
 // Scan form of the tensor-core path.  Automatic choice: the chunk-wise scans
@@ -1746,7 +2203,8 @@ inline bool use_chunk_scan(int form, size_t BH, int T, int chunk, int NC, int sm
 
 // Kernel launches of one forward on the tensor-core path (without the decay
 // bridge): the chunk-wise scans take two.
-inline int tc_launches_per_forward(int form, size_t BH, int T, int chunk, int NC) {
+inline int tc_launches_per_forward(int d, int form, size_t BH, int T, int chunk, int NC) {
+  if (d != 128) return 4;   // d = 64: Gram, inverse, paired-chain scans, readout
   return use_chunk_scan(form, BH, T, chunk, NC, tc::num_sms()) ? 5 : 4;
 }
 
@@ -1793,8 +2251,77 @@ int launch_tc(size_t BH, int T, int U, int chunk, int NC, int window, const vda_
   }
   const float eps = a.eps > 0.f ? a.eps : 1e-6f;
   timer.begin(3, s);
-  if ((rc = tc::launch_readout(a.q, a.gate, a.rms_weight, st, bridge, a.out, BH, T, U, chunk, NC, window, eps,
+  if ((rc = tc::launch_readout<128>(a.q, a.gate, a.rms_weight, st, bridge, a.out, BH, T, U, chunk, NC, window, eps,
                                s)) != VDA_OK)
+    return rc;
+  timer.end(3, s);
+  return debug_check("readout", s);
+}
+
+// The d = 64 schedule: Gram kernel (operands swapped, M = 128), the FP32
+// Gauss-Jordan inverse (which also writes the scan's operand image), the
+// paired-chain scans, decay bridge (with a decay gate), readout.
+template <typename Timer>
+int launch_tc64(size_t BH, int T, int U, int chunk, int NC, int window, const vda_args& a, char* ws_AM,
+                char* ws_B, char* ws_states, char* ws_img, char* ws_bridge, cudaStream_t s, float* stats_out,
+                Timer& timer) {
+  constexpr int D = 64;
+  const size_t FH = BH * (size_t)T;
+  const size_t fdd = FH * (size_t)D * D;
+  float* AM = reinterpret_cast<float*>(ws_AM);
+  float* Bt = reinterpret_cast<float*>(ws_B);
+  float* st = reinterpret_cast<float*>(ws_states);
+  uint8_t* img = reinterpret_cast<uint8_t*>(ws_img);
+  int rc;
+  {
+    CUtensorMap tmK, tmV;
+    if (!tc::encode_bf16_3d(&tmK, a.k, (uint64_t)U, FH, 64, D) || !tc::encode_bf16_3d(&tmV, a.v, (uint64_t)U, FH, 64, D))
+      return VDA_ERR_CUDA;
+    if (cudaFuncSetAttribute(tc::k_stats64_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tc::Stats64Cfg::SMEM) != cudaSuccess)
+      return launch_status("k_stats64_tc (shared-memory attribute)");
+    const size_t sms = (size_t)tc::num_sms();
+    const size_t rounds = (FH + sms - 1) / sms;
+    const int grid = (int)((FH + rounds - 1) / rounds);
+    timer.begin(0, s);
+    rc = tc::launch_pdl("k_stats64_tc", tc::k_stats64_tc, dim3(grid), dim3(tc::Stats64Cfg::THREADS),
+                        tc::Stats64Cfg::SMEM, s, tmK, tmV, a.beta, U, (int)FH, AM, Bt,
+                        stats_out ? stats_out + fdd : nullptr);
+    if (rc != VDA_OK) return rc;
+    timer.end(0, s);
+  }
+  if ((rc = debug_check("stats", s)) != VDA_OK) return rc;
+  if (stats_out && cudaMemcpyAsync(stats_out, AM, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return VDA_ERR_CUDA;
+  timer.begin(1, s);
+  k_gj_inverse<D><<<(unsigned)FH, 256, 0, s>>>(AM, img);
+  if ((rc = launch_status("k_gj_inverse")) != VDA_OK) return rc;
+  timer.end(1, s);
+  if ((rc = debug_check("inverse", s)) != VDA_OK) return rc;
+  if (stats_out &&
+      cudaMemcpyAsync(stats_out + 2 * fdd, AM, fdd * sizeof(float), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return VDA_ERR_CUDA;
+  if (cudaFuncSetAttribute(tc::k_scan64_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)tc::Scan64Cfg::SMEM) != cudaSuccess)
+    return VDA_ERR_CUDA;
+  timer.begin(2, s);
+  rc = tc::launch_pdl("k_scan64_tc", tc::k_scan64_tc, dim3((unsigned)BH), dim3(tc::Scan64Cfg::THREADS),
+                      tc::Scan64Cfg::SMEM, s, (const uint8_t*)img, (const float*)Bt, a.S0_fwd, a.S0_rev, a.alpha,
+                      st, (int)BH, T, chunk, NC);
+  if (rc != VDA_OK) return rc;
+  timer.end(2, s);
+  if ((rc = debug_check("scan", s)) != VDA_OK) return rc;
+  float* bridge = nullptr;
+  if (a.alpha) {
+    bridge = reinterpret_cast<float*>(ws_bridge);
+    const size_t n = FH * (size_t)D;
+    k_decay_bridge<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.alpha, (int)BH, T, D, chunk, window, bridge);
+    if ((rc = launch_status("k_decay_bridge")) != VDA_OK) return rc;
+  }
+  const float eps = a.eps > 0.f ? a.eps : 1e-6f;
+  timer.begin(3, s);
+  if ((rc = tc::launch_readout<D>(a.q, a.gate, a.rms_weight, st, bridge, a.out, BH, T, U, chunk, NC, window, eps,
+                                  s)) != VDA_OK)
     return rc;
   timer.end(3, s);
   return debug_check("readout", s);

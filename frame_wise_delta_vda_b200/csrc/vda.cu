@@ -69,7 +69,7 @@ Plan make_plan(int B, int H, int T, int U, int d, int chunk, int window, int dty
   // chunk maps of the chunk-wise scans (tensor-core path): in A's region,
   // which the scans no longer need, when they fit there
   p.off_maps = p.off_AM;
-  if (p.tc) {
+  if (p.tc && d == 128) {
     const size_t maps = vda::tc::chunk_maps_bytes(p.BH, p.NC);
     if (maps > p.FH * dd) {
       p.off_maps = off;
@@ -153,7 +153,7 @@ int launch_simt(const Plan& p, const vda_args& a, char* ws, cudaStream_t s, Call
       return VDA_ERR_CUDA;
   }
   tm.begin(1, s);
-  vda::k_gj_inverse<D><<<(unsigned)p.FH, 256, 0, s>>>(AM);
+  vda::k_gj_inverse<D><<<(unsigned)p.FH, 256, 0, s>>>(AM, nullptr);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
   tm.end(1, s);
   if (stats_out) {
@@ -228,7 +228,11 @@ int forward_impl(const vda_args& a, char* ws, const Plan& p, float* states_out, 
   CallTimer tm;
   tm.slot = timing_begin_call();
   int rc;
-  if (p.tc) {
+  if (p.tc && p.d == 64) {
+    rc = vda::launch_tc64(p.BH, p.T, p.U, p.chunk, p.NC, p.window, a, ws + p.off_AM, ws + p.off_B,
+                          ws + p.off_states, ws + p.total - vda::tc_extra_workspace_bytes(true, p.FH, p.d),
+                          ws + p.off_bridge, s, stats_out, tm);
+  } else if (p.tc) {
     rc = vda::launch_tc(p.BH, p.T, p.U, p.chunk, p.NC, p.window, a, ws + p.off_AM, ws + p.off_B,
                         ws + p.off_states, ws + p.total - vda::tc_extra_workspace_bytes(true, p.FH, p.d),
                         ws + p.off_bridge, ws + p.off_maps, s, stats_out, tm);
@@ -268,7 +272,7 @@ int text_state_simt(const Plan& p, const void* k, const void* v, const float* be
   vda::k_stats_simt<D, TIo><<<(unsigned)p.FH, 256, 0, s>>>(static_cast<const TIo*>(k),
                                                            static_cast<const TIo*>(v), beta, p.U, AM, Bm);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
-  vda::k_gj_inverse<D><<<(unsigned)p.FH, 256, 0, s>>>(AM);
+  vda::k_gj_inverse<D><<<(unsigned)p.FH, 256, 0, s>>>(AM, nullptr);
   if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
   dim3 gs((unsigned)p.BH, 1, D / 16);
   vda::k_scan_simt<D, 16><<<gs, D, 0, s>>>(AM, Bm, nullptr, nullptr, nullptr, st, (int)p.BH, 1, 1, p.NC);
@@ -290,7 +294,7 @@ int text_state_dispatch(const Plan& p, const void* k, const void* v, const float
 
 int text_state_impl(const Plan& p, const void* k, const void* v, const float* beta, char* ws,
                     cudaStream_t s) {
-  if (p.tc)
+  if (p.tc && p.d == 128)
     return vda::tc_text_state(p.BH, p.U, k, v, beta, ws + p.off_AM, ws + p.off_B, ws + p.off_states,
                               ws + p.total - vda::tc_extra_workspace_bytes(true, p.FH, p.d), s);
   return p.dtype == VDA_BF16 ? text_state_dispatch<__nv_bfloat16>(p, k, v, beta, ws, s)
@@ -440,7 +444,7 @@ size_t vda_workspace_bytes(int B, int H, int T, int U, int d_k, int d_v, int chu
 int vda_launches_per_forward(int B, int H, int T, int U, int d_k, int d_v, int chunk, int dtype) {
   if (check_sizes(B, H, T, U, d_k, d_v, chunk, 0, dtype) != VDA_OK) return 0;
   const Plan p = make_plan(B, H, T, U, d_k, chunk, 0, dtype);
-  return p.tc ? vda::tc_launches_per_forward(VDA_SCAN_AUTO, p.BH, p.T, p.chunk, p.NC) : 4;
+  return p.tc ? vda::tc_launches_per_forward(p.d, VDA_SCAN_AUTO, p.BH, p.T, p.chunk, p.NC) : 4;
 }
 
 int vda_forward_ex(const vda_args* args, void* workspace, size_t workspace_bytes,

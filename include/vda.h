@@ -48,8 +48,9 @@
  *     vda_forward_f32 have no decay (alpha = 1); vda_forward_ex,
  *     vda_forward_host and vda_forward_noalloc take it from vda_args.
  *   - Supported sizes: d_k == d_v in {16, 32, 64, 128}; chunk >= 1;
- *     window_chunks >= 0; B, H, T, U >= 1.  d = 128 with bf16 I/O runs on the
- *     tcgen05 tensor-core kernels; the other sizes run on SIMT kernels.
+ *     window_chunks >= 0; B, H, T, U >= 1.  d = 128 and d = 64 with bf16 I/O
+ *     run on the tcgen05 tensor-core kernels (at d = 64 with the FP32
+ *     Gauss-Jordan inverse); the other sizes run on SIMT kernels.
  *   - Errors: every argument is validated before any launch; no exception
  *     crosses the ABI.  See vda_status.
  */
@@ -84,7 +85,7 @@ typedef enum vda_dtype {
 } vda_dtype;
 
 /* How the forward and reverse scans of Section 2.2 run on the tensor-core
- * path (d = 128, bf16); the SIMT path always scans frame by frame.  Both give
+ * path at d = 128 (bf16); the other paths always scan frame by frame.  Both give
  * the same boundary states up to rounding.
  *   VDA_SCAN_FRAMES: one sequential chain of T frame updates per (b, h,
  *     direction), S <- (S Diag(alpha_t) + B_t) M_t.
