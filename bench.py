@@ -44,6 +44,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # ----------------------------------------------------------------------------
+L2_BYTES = 126 * 1024 * 1024
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -320,7 +323,9 @@ def run_prep(args):
             "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"{pw.name}: B={pw.B} H={pw.H} T={pw.T} grid={pw.Hl}x{pw.Wl} d={pw.d}",
-                       "l2": "inputs larger than L2 (2.2 GB read per step), no flush"},
+                       "l2": (f"inputs larger than L2 ({3 * pw.B * pw.T * pw.U * pw.H * pw.d * 2 / 1e9:.2f} GB read "
+                              "per step), no flush" if 3 * pw.B * pw.T * pw.U * pw.H * pw.d * 2 > 2 * L2_BYTES else
+                              "inputs fit in L2: read back from L2 between steps (not a roofline number)")},
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / peaks["hbm_gbs"], "traffic": None, "kernel": "k_prep_kv + k_prep_q",
                          "algorithmic_per_launch": byts, "peak_source": f"hbm_gbs ({peak_src})"},
@@ -427,21 +432,38 @@ def main():
     torch.cuda.synchronize()
     assert api.vda_device_status() == 0
 
+    # inputs smaller than twice the L2 (126 MB) would be served from L2 on the
+    # next step: then a 256 MB buffer is written before every step and each
+    # step is timed alone
+    in_bytes = algorithmic(wl_rank)["op"]["bytes"]
+    flush = in_bytes < 2 * L2_BYTES
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
     sampler = ClockSampler(local_rank)
     sampler.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
+    if flush:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for k, (e0, e1) in enumerate(evs):
+            flush_buf.fill_(k & 0xFF)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / args.steps
+    else:
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        ms = ev0.elapsed_time(ev1) / args.steps
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms = ev0.elapsed_time(ev1) / args.steps
     # per-kernel device time: further steps of the same workload with CUDA
     # events just before and after each launch, on its stream (kept out of the
     # region above, so that the headline time carries no extra stream work)
@@ -474,7 +496,7 @@ def main():
         dist.destroy_process_group()
     if rank != 0:
         return
-    emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches, wl_rank=wl_rank)
+    emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches, wl_rank=wl_rank, flushed=flush)
 
 
 def run_e2e(api, x, S0, out, wl, dev, e2e_steps, world, dist):
@@ -511,7 +533,7 @@ def run_e2e(api, x, S0, out, wl, dev, e2e_steps, world, dist):
     return {"e2e_s": e2e_s, "h2d": h2d, "d2h": d2h}
 
 
-def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches, wl_rank=None):
+def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches, wl_rank=None, flushed=False):
     """The JSON line.  wl: the workload of the metric (each rank's own problem
     with replicas, the one sharded problem with heads); wl_rank: the problem
     one rank's kernels process (for the roofline)."""
@@ -555,7 +577,10 @@ def emit(args, wl, world, ms_max, stage_ms, calls, clocks, e2e, launches, wl_ran
                                   else ""),
                    "per_rank_problem": (f"token shard of one problem, {wl_rank.H} heads per GPU after the "
                                         "all-to-all" if heads else "independent problem of the same size per GPU"),
-                   "l2": "inputs larger than L2 (about 3 GB read per step), no flush",
+                   "l2": (f"inputs of {alg['op']['bytes'] / 1e6:.0f} MB fit in L2 (126 MB): a 256 MB buffer is "
+                          "written before every step and each step is timed alone" if flushed else
+                          f"inputs larger than L2 ({alg['op']['bytes'] / 1e9:.1f} GB read and written per step), "
+                          "no flush"),
                    "kernel_timing": f"events around each launch over {calls} further steps of this workload; "
                                     "ms_per_step is timed without them",
                    "parallelism": f"heads{world} (all-to-all)" if heads else f"replicas{world}",

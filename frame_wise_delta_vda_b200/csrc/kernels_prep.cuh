@@ -30,39 +30,60 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float2 v) {
 
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
-constexpr int kThreads = 256;
-constexpr int kMaxWc = 16;   // grid columns per thread
+constexpr int kThreads = 512;
+constexpr int kMaxNxt = 8;   // grid columns per thread
 
-// Shared memory of k_prep_kv: staged input rows (bf16) and the ring of the
-// last five frames' spatial results (bf16 pairs); the output row for the L2
-// reduction (fp32) reuses the staging area once the spatial filter is done.
-// 20 bytes per column and channel, so two CTAs fit on an SM.
-__host__ __device__ constexpr size_t kv_smem_bytes(int Wl, int D) {
-  return (size_t)Wl * D * (5 * 2 + 5 * 2);
+// 16-B asynchronous global -> shared copy (L1 bypassed) and its groups
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Geometry of k_prep_kv: thread = (channel pair, column slice); NS slices of
+// NXT grid columns each; the staged rows carry two zero columns on each side
+// (x = -2 .. NS * NXT + 1), so the spatial filter needs no bounds checks.
+__host__ __device__ constexpr int kv_slices(int D) { return kThreads / (D / 2); }
+__host__ __device__ constexpr int kv_cols_per_thread(int Wl, int D) { return (Wl + kv_slices(D) - 1) / kv_slices(D); }
+__host__ __device__ constexpr size_t kv_stage_bytes(int Wl, int D) {
+  return (size_t)5 * (kv_slices(D) * kv_cols_per_thread(Wl, D) + 4) * D * 2;
+}
+// Shared memory: nst staging buffers of rows y-2..y+2 (bf16 pairs), the ring
+// of the last five frames' spatial results (bf16 pairs) and the fp32 output
+// row of the L2 normalisation.
+__host__ __device__ constexpr size_t kv_smem_bytes(int Wl, int D, int nst) {
+  return (size_t)nst * kv_stage_bytes(Wl, D) + (size_t)5 * Wl * D * 2 + (size_t)Wl * D * 4;
 }
 
 // One CTA per (grid row y, batch-head, tensor K or V).  It walks the frames:
-// for each input frame it stages rows y-2..y+2, computes the spatial filter
-// for row y into a five-frame ring, and, two frames behind, the temporal
-// filter, SiLU and (K only) the L2 normalisation of output frame t.  Thread =
-// (channel pair cp, column slice xs): channel pairs use packed fp32 FMAs.
-template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+// the rows y-2..y+2 of a frame arrive by cp.async one frame ahead (two
+// staging buffers when they fit, else one, refilled once the spatial filter
+// has read it); the spatial filter of row y goes into a five-frame ring, and,
+// two frames behind, the temporal filter, SiLU and (K only) the L2
+// normalisation of output frame t.  Thread = (channel pair cp, column slice
+// xs): channel pairs use packed fp32 FMAs, and each thread keeps its NXT
+// columns' accumulators and the 5-tap window of one staged row in registers.
+template <int D, int NXT>
+__global__ void __launch_bounds__(kThreads, 1)
 k_prep_kv(const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict__ vin,
           const float* __restrict__ wk_s, const float* __restrict__ wk_t,
           const float* __restrict__ wv_s, const float* __restrict__ wv_t,
           __nv_bfloat16* __restrict__ kout, __nv_bfloat16* __restrict__ vout,
-          int H, int T, int Hl, int Wl, float eps) {
+          int H, int T, int Hl, int Wl, float eps, int nst) {
   constexpr int NP = D / 2;              // channel pairs
   constexpr int NS = kThreads / NP;      // column slices
+  constexpr int WS = NS * NXT + 4;       // staged columns
+  constexpr int V8 = D / 8;              // 16-B chunks per token
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint32_t* stage = reinterpret_cast<uint32_t*>(smem_raw);                      // [5][Wl][NP] bf16 pairs
-  uint32_t* ring = reinterpret_cast<uint32_t*>(smem_raw + (size_t)5 * Wl * D * 2);  // [5][Wl][NP] bf16 pairs
-  float* tile = reinterpret_cast<float*>(smem_raw);                                // [Wl][D], over the stage
+  const size_t stage_words = (size_t)5 * WS * NP;
+  uint32_t* stage0 = reinterpret_cast<uint32_t*>(smem_raw);                  // [nst][5][WS][NP]
+  uint32_t* ring = stage0 + (size_t)nst * stage_words;                       // [5][Wl][NP]
+  float* tile = reinterpret_cast<float*>(ring + (size_t)5 * Wl * NP);        // [Wl][D]
 
   const int y = blockIdx.x, bh = blockIdx.y, isv = blockIdx.z;
-  const int Hn = H;
-  const int b = bh / Hn, h = bh - (bh / Hn) * Hn;
+  const int b = bh / H, h = bh - (bh / H) * H;
   const __nv_bfloat16* in = isv ? vin : kin;
   __nv_bfloat16* out = isv ? vout : kout;
   const float* ws = (isv ? wv_s : wk_s) + (size_t)h * D * 25;
@@ -70,8 +91,7 @@ k_prep_kv(const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict
   const int U = Hl * Wl;
   const int tid = threadIdx.x, cp = tid % NP, xs = tid / NP;
   const int c0 = 2 * cp;
-  const int Wc = (Wl + NS - 1) / NS;
-  const int xb = xs * Wc, nx = max(0, min(Wc, Wl - xb));
+  const int xb = xs * NXT;
 
   float2 wsp[25], wtp[5];
 #pragma unroll
@@ -79,81 +99,82 @@ k_prep_kv(const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict
 #pragma unroll
   for (int s = 0; s < 5; ++s) wtp[s] = make_float2(__ldg(wt + (size_t)c0 * 5 + s), __ldg(wt + (size_t)(c0 + 1) * 5 + s));
 
-  const size_t tok_stride = (size_t)Hn * D;   // elements between consecutive tokens of the input
-  for (int tin = 0; tin < T + 2; ++tin) {
-    __syncthreads();   // the previous frame's stage and ring reads are done
-    if (tin < T) {
-      // stage rows y-2..y+2 of frame tin (zero outside the grid): 16-B vectors
-      constexpr int V8 = D / 8;
-      const size_t frame_tok = ((size_t)b * T + tin) * U;
+  // padding columns and rows outside the grid are never loaded: zero them once
+  for (size_t e = tid; e < (size_t)nst * stage_words; e += kThreads) stage0[e] = 0u;
+  __syncthreads();
+
+  const size_t tok_stride = (size_t)H * D;   // elements between consecutive tokens of the input
+  auto issue = [&](int f) {   // rows y-2..y+2 of frame f -> staging buffer f % nst
+    uint32_t* st = stage0 + (size_t)(f % nst) * stage_words;
+    const __nv_bfloat16* fbase = in + ((size_t)b * T + f) * U * tok_stride + (size_t)h * D;
+#pragma unroll 1
+    for (int r = 0; r < 5; ++r) {
+      const int row = y + r - 2;
+      if (row < 0 || row >= Hl) continue;   // stays zero
+      const __nv_bfloat16* rbase = fbase + (size_t)row * Wl * tok_stride;
+      uint32_t* srow = st + ((size_t)r * WS + 2) * NP;
       for (int e = tid; e < Wl * V8; e += kThreads) {
-        const int v8 = e % V8, x = e / V8;   // V8 is a power of two
-#pragma unroll
-        for (int r = 0; r < 5; ++r) {
-          const int row = y + r - 2;
-          uint4 val = make_uint4(0u, 0u, 0u, 0u);
-          if (row >= 0 && row < Hl) {
-            const size_t tok = frame_tok + (size_t)row * Wl + x;
-            val = __ldg(reinterpret_cast<const uint4*>(in + tok * tok_stride + (size_t)h * D) + v8);
-          }
-          reinterpret_cast<uint4*>(stage)[((size_t)r * Wl + x) * V8 + v8] = val;
-        }
+        const int v8 = e & (V8 - 1), x = e / V8;   // V8 is a power of two
+        cp_async16(srow + (size_t)x * NP + v8 * 4, rbase + (size_t)x * tok_stride + v8 * 8);
       }
     }
-    __syncthreads();
-    // spatial filter of row y for this thread's columns and channel pair
-    uint32_t* ring_t = ring + (size_t)(tin % 5) * Wl * NP;
-    if (tin < T) {
-      float2 acc[kMaxWc];
+    cp_async_commit();
+  };
+  issue(0);
+  if (nst == 2 && T > 1) issue(1);
+
+  for (int f = 0; f < T + 2; ++f) {
+    if (f < T) {   // this frame's rows have landed (the next frame's may still be in flight)
+      if (nst == 2 && f + 1 < T) cp_async_wait<1>();
+      else cp_async_wait<0>();
+    }
+    __syncthreads();   // ... for every thread; the previous frame's ring and tile reads are done
+    uint32_t* ring_t = ring + (size_t)(f % 5) * Wl * NP;
+    if (f < T) {
+      const uint32_t* st = stage0 + (size_t)(f % nst) * stage_words + cp;
+      float2 acc[NXT];
 #pragma unroll
-      for (int xi = 0; xi < kMaxWc; ++xi) acc[xi] = make_float2(0.f, 0.f);
+      for (int i = 0; i < NXT; ++i) acc[i] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int dy = 0; dy < 5; ++dy) {
         const int row = y + dy - 2;
-        if (row < 0 || row >= Hl) continue;
-        const uint32_t* srow = stage + (size_t)dy * Wl * NP + cp;
-        auto at = [&](int x) -> float2 {
-          return (x >= 0 && x < Wl) ? bf2_to_f2(srow[(size_t)x * NP]) : make_float2(0.f, 0.f);
-        };
-        float2 w0 = at(xb - 2), w1 = at(xb - 1), w2 = at(xb), w3 = at(xb + 1), w4 = at(xb + 2);
+        if (row < 0 || row >= Hl) continue;   // a zero row
+        const uint32_t* srow = st + (size_t)dy * WS * NP + (size_t)xb * NP;
+        float2 win[NXT + 4];
 #pragma unroll
-        for (int xi = 0; xi < kMaxWc; ++xi) {
-          if (xi < nx) {
-            float2 a = acc[xi];
-            a = ffma2(wsp[dy * 5 + 0], w0, a);
-            a = ffma2(wsp[dy * 5 + 1], w1, a);
-            a = ffma2(wsp[dy * 5 + 2], w2, a);
-            a = ffma2(wsp[dy * 5 + 3], w3, a);
-            a = ffma2(wsp[dy * 5 + 4], w4, a);
-            acc[xi] = a;
-            w0 = w1; w1 = w2; w2 = w3; w3 = w4;
-            w4 = at(xb + xi + 3);
-          }
+        for (int q = 0; q < NXT + 4; ++q) win[q] = bf2_to_f2(srow[(size_t)q * NP]);
+#pragma unroll
+        for (int i = 0; i < NXT; ++i) {
+          float2 a = acc[i];
+#pragma unroll
+          for (int dx = 0; dx < 5; ++dx) a = ffma2(wsp[dy * 5 + dx], win[i + dx], a);
+          acc[i] = a;
         }
       }
 #pragma unroll
-      for (int xi = 0; xi < kMaxWc; ++xi)
-        if (xi < nx) ring_t[(size_t)(xb + xi) * NP + cp] = f2_to_bf2(acc[xi]);
+      for (int i = 0; i < NXT; ++i)
+        if (xb + i < Wl) ring_t[(size_t)(xb + i) * NP + cp] = f2_to_bf2(acc[i]);
     } else {
       // frames past the clip contribute zero (temporal zero padding)
 #pragma unroll
-      for (int xi = 0; xi < kMaxWc; ++xi)
-        if (xi < nx) ring_t[(size_t)(xb + xi) * NP + cp] = 0u;
+      for (int i = 0; i < NXT; ++i)
+        if (xb + i < Wl) ring_t[(size_t)(xb + i) * NP + cp] = 0u;
     }
-    __syncthreads();
-    if (tin < 2) continue;
-    // temporal filter, SiLU of output frame tout = tin - 2
-    const int tout = tin - 2;
+    __syncthreads();   // ring slot written; this frame's staging buffer has been read
+    if (f + nst < T) issue(f + nst);
+    if (f < 2) continue;
+    // temporal filter, SiLU of output frame tout = f - 2
+    const int tout = f - 2;
 #pragma unroll
-    for (int xi = 0; xi < kMaxWc; ++xi) {
-      if (xi >= nx) continue;
-      const int x = xb + xi;
+    for (int i = 0; i < NXT; ++i) {
+      const int x = xb + i;
+      if (x >= Wl) continue;
       float2 o = make_float2(0.f, 0.f);
 #pragma unroll
       for (int s = 0; s < 5; ++s) {
-        const int f = tout + s - 2;
-        if (f < 0) continue;   // frames before the clip: zero padding
-        o = ffma2(wtp[s], bf2_to_f2(ring[((size_t)(f % 5) * Wl + x) * NP + cp]), o);
+        const int fr = tout + s - 2;
+        if (fr < 0) continue;   // frames before the clip: zero padding
+        o = ffma2(wtp[s], bf2_to_f2(ring[((size_t)(fr % 5) * Wl + x) * NP + cp]), o);
       }
       o.x = silu(o.x);
       o.y = silu(o.y);

@@ -375,18 +375,37 @@ int noalloc_scratch(char** out) {
 
 // ============================================================================
 namespace {
+template <int D, int NXT>
+int launch_prep_kv(const vda_prep_args& a, int nst, cudaStream_t s, float eps) {
+  using namespace vda::prep;
+  const size_t smem = kv_smem_bytes(a.Wl, D, nst);
+  if (cudaFuncSetAttribute(k_prep_kv<D, NXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return VDA_ERR_CUDA;
+  k_prep_kv<D, NXT><<<dim3((unsigned)a.Hl, (unsigned)(a.B * a.H), 2), kThreads, smem, s>>>(
+      static_cast<const __nv_bfloat16*>(a.k_in), static_cast<const __nv_bfloat16*>(a.v_in), a.wk_s, a.wk_t, a.wv_s,
+      a.wv_t, static_cast<__nv_bfloat16*>(a.k_out), static_cast<__nv_bfloat16*>(a.v_out), a.H, a.T, a.Hl, a.Wl, eps,
+      nst);
+  return cudaGetLastError() == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+}
+
 template <int D>
-int launch_prep(const vda_prep_args& a) {
+int launch_prep(const vda_prep_args& a, int nst) {
   using namespace vda::prep;
   cudaStream_t s = static_cast<cudaStream_t>(a.stream);
-  const size_t smem = kv_smem_bytes(a.Wl, D);
   const float eps = a.eps > 0.f ? a.eps : 1e-6f;
-  if (cudaFuncSetAttribute(k_prep_kv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return VDA_ERR_CUDA;
-  k_prep_kv<D><<<dim3((unsigned)a.Hl, (unsigned)(a.B * a.H), 2), kThreads, smem, s>>>(
-      static_cast<const __nv_bfloat16*>(a.k_in), static_cast<const __nv_bfloat16*>(a.v_in), a.wk_s, a.wk_t, a.wv_s,
-      a.wv_t, static_cast<__nv_bfloat16*>(a.k_out), static_cast<__nv_bfloat16*>(a.v_out), a.H, a.T, a.Hl, a.Wl, eps);
-  if (cudaGetLastError() != cudaSuccess) return VDA_ERR_CUDA;
+  int rc = VDA_ERR_UNSUPPORTED;
+  switch (kv_cols_per_thread(a.Wl, D)) {
+    case 1: rc = launch_prep_kv<D, 1>(a, nst, s, eps); break;
+    case 2: rc = launch_prep_kv<D, 2>(a, nst, s, eps); break;
+    case 3: rc = launch_prep_kv<D, 3>(a, nst, s, eps); break;
+    case 4: rc = launch_prep_kv<D, 4>(a, nst, s, eps); break;
+    case 5: rc = launch_prep_kv<D, 5>(a, nst, s, eps); break;
+    case 6: rc = launch_prep_kv<D, 6>(a, nst, s, eps); break;
+    case 7: rc = launch_prep_kv<D, 7>(a, nst, s, eps); break;
+    case 8: rc = launch_prep_kv<D, 8>(a, nst, s, eps); break;
+  }
+  if (rc != VDA_OK) return rc;
   const size_t warps = (size_t)a.B * a.T * a.Hl * a.Wl * a.H;
   const size_t blocks = (warps * 32 + 255) / 256;
   k_prep_q<D><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.q_in),
@@ -407,20 +426,22 @@ int vda_prep(const vda_prep_args* a) {
     if (!ptr || !aligned16(ptr)) return VDA_ERR_INVALID_ARGUMENT;
   const int d = a->d;
   if (d != 16 && d != 32 && d != 64 && d != 128) return VDA_ERR_UNSUPPORTED;
-  const int ns = vda::prep::kThreads / (d / 2);
-  if ((a->Wl + ns - 1) / ns > vda::prep::kMaxWc) return VDA_ERR_UNSUPPORTED;
+  if (vda::prep::kv_cols_per_thread(a->Wl, d) > vda::prep::kMaxNxt) return VDA_ERR_UNSUPPORTED;
   int dev = 0, max_smem = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
     return VDA_ERR_CUDA;
-  if (vda::prep::kv_smem_bytes(a->Wl, d) > (size_t)max_smem) return VDA_ERR_UNSUPPORTED;
+  // two staging buffers (the next frame's rows load during this frame's
+  // filters) when they fit, else one
+  const int nst = vda::prep::kv_smem_bytes(a->Wl, d, 2) <= (size_t)max_smem ? 2 : 1;
+  if (vda::prep::kv_smem_bytes(a->Wl, d, nst) > (size_t)max_smem) return VDA_ERR_UNSUPPORTED;
   if ((double)a->B * a->H * a->T * a->Hl * a->Wl * d > 4.0e12 || (double)a->B * a->H > 65535.0 || a->Hl > 2147483647)
     return VDA_ERR_UNSUPPORTED;
   switch (d) {
-    case 16: return launch_prep<16>(*a);
-    case 32: return launch_prep<32>(*a);
-    case 64: return launch_prep<64>(*a);
-    default: return launch_prep<128>(*a);
+    case 16: return launch_prep<16>(*a, nst);
+    case 32: return launch_prep<32>(*a, nst);
+    case 64: return launch_prep<64>(*a, nst);
+    default: return launch_prep<128>(*a, nst);
   }
 }
 
@@ -557,6 +578,14 @@ int vda_forward_host(const vda_args* ha, void* device_buffer, size_t device_byte
   const size_t BH = (size_t)ha->B * ha->H;
   const size_t per_head_tok = (size_t)ha->T * ha->U;
   const int d = ha->d_k;
+  // the scan form the whole problem would take, so that every head group
+  // computes what vda_forward_ex computes for all heads at once
+  int scan_form = ha->scan_form;
+  if (scan_form == VDA_SCAN_AUTO)
+    scan_form = vda::use_chunk_scan(VDA_SCAN_AUTO, BH, ha->T, ha->chunk, (ha->T + ha->chunk - 1) / ha->chunk,
+                                    vda::tc::num_sms())
+                    ? VDA_SCAN_CHUNKS
+                    : VDA_SCAN_FRAMES;
 #define VDA_CK(x) do { if ((x) != cudaSuccess) return VDA_ERR_CUDA; } while (0)
   // the copy / compute pipeline; on an error it returns at once, with copies
   // possibly still queued on the three streams
@@ -592,6 +621,7 @@ int vda_forward_host(const vda_args* ha, void* device_buffer, size_t device_byte
     if (g >= 2) VDA_CK(cudaStreamWaitEvent(P->comp, P->out_done[sl], 0));
     vda_args a = *ha;
     a.B = 1; a.H = nh;
+    a.scan_form = scan_form;
     a.q = S + L.slot_off_q; a.k = S + L.slot_off_k; a.v = S + L.slot_off_v; a.gate = S + L.slot_off_g;
     a.beta = reinterpret_cast<const float*>(S + L.slot_off_beta);
     a.rms_weight = d_w;

@@ -172,9 +172,11 @@ VDA_API int vda_text_state(int dtype, const void* k_text, const void* v_text, co
  * gate, rms_weight, S0_fwd, S0_rev, out) is a host pointer (page-locked for
  * overlap); the call copies the inputs to the device, runs the forward and
  * copies `out` back, pipelining groups of heads over two streams (copy and
- * compute) so that transfers overlap the kernels.  `device_buffer` is caller
- * device memory of at least vda_forward_host_bytes() bytes (256-byte
- * aligned).  Synchronous: returns when `out` is complete on the host. */
+ * compute) so that transfers overlap the kernels.  Every group takes the
+ * scan form the whole problem takes, so `out` equals vda_forward_ex's bit for
+ * bit.  `device_buffer` is caller device memory of at least
+ * vda_forward_host_bytes() bytes (256-byte aligned).  Synchronous: returns
+ * when `out` is complete on the host. */
 VDA_API size_t vda_forward_host_bytes(int B, int H, int T, int U, int d_k, int d_v,
                               int chunk, int dtype);
 VDA_API int vda_forward_host(const vda_args* host_args, void* device_buffer, size_t device_bytes);
@@ -247,9 +249,11 @@ VDA_API int vda_launches_per_forward(int B, int H, int T, int U, int d_k, int d_
  *                     video tokens, heads inner; token u = y * Wl + x)
  *   wk_s, wv_s        [H, d, 5, 5] float32, wk_t, wv_t [H, d, 5] float32
  *   q_out, k_out, v_out [B, H, T, U, d] bf16 (the layout vda_forward reads)
- * Supported: bf16, d in {16, 32, 64, 128}, Wl * d * 20 bytes of shared
- * memory within the device limit and at most 16 grid columns per thread
- * slice (Wl <= 64 at d = 128).  Inputs and outputs must not overlap.
+ * Supported: bf16, d in {16, 32, 64, 128}, at most 8 grid columns per
+ * thread slice (Wl <= 8 * 1024 / d) and the staging rows, the five-frame ring
+ * and one fp32 output row (about (5 (Wl + 4) + 5 Wl + 2 Wl) * 2 d bytes)
+ * within the device's shared memory (Wl <= 64 at d = 128).  Inputs and
+ * outputs must not overlap.
  * Returns vda_status. */
 typedef struct vda_prep_args {
   const void* q_in;

@@ -113,6 +113,18 @@ def test_launch_count(L):
     assert L.vda_launches_per_forward(1, 6, 60, 1008, 128, 128, 1, 0) == 4   # one-frame chunks
 
 
+def test_d64_tensor_core_workspace(L):
+    # d = 64, bf16: the tensor-core path adds the scan's operand images
+    # (16 KB per frame-head) to A/M, B and the boundary states; fp32 I/O at
+    # d = 64 runs the SIMT path without them
+    fh, dd = 8 * 20, 64 * 64 * 4
+    bf16 = L.vda_workspace_bytes(1, 8, 20, 240, 64, 64, 5, 0)
+    f32 = L.vda_workspace_bytes(1, 8, 20, 240, 64, 64, 5, 1)
+    assert bf16 - f32 == fh * 16384
+    assert f32 >= 2 * fh * dd + 2 * 8 * 5 * dd
+    assert L.vda_launches_per_forward(1, 8, 20, 240, 64, 64, 5, 0) == 4
+
+
 def test_chunk_maps_fit_the_workspace(L):
     # the chunk maps (J_c fp32 + P_c image, 128 KB per direction and chunk)
     # live in A's region when 4 NC <= T, else in a region of their own

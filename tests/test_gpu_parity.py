@@ -197,9 +197,14 @@ def test_scan_is_non_expansive_on_device():
 
 
 # --- the host-buffer entry point and determinism ------------------------------
-def test_forward_host_matches_device_path_bitwise():
+@pytest.mark.parametrize("name", ["small", "corr"])
+def test_forward_host_matches_device_path_bitwise(name):
+    """The host-buffer entry runs the heads in groups; each group takes the
+    scan form the whole problem takes (at 16 heads the per-frame scans, while
+    a group of 2 heads alone would take the chunk-wise ones), so the result
+    is the device entry's bit for bit."""
     api = _api()
-    wl = gen.WORKLOADS["small"]
+    wl = gen.WORKLOADS[name]
     x = gen.make_inputs(wl)
     t = _device_inputs(wl, x)
     out_dev, _, _ = _run(wl, t)
