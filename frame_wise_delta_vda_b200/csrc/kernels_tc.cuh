@@ -1085,7 +1085,7 @@ struct ScanArgs {
 
 struct ScanCfg {
   static constexpr int THREADS = 320;
-  static constexpr int PREFETCH = 3;                       // steps of L2 prefetch lead
+  static constexpr int PREFETCH = 1;                       // steps of L2 prefetch lead (1 measured best)
   static constexpr int WARP_PROD = 8;
   static constexpr int WARP_MMA = 9;
   static constexpr uint32_t OFF_M = 0;                    // 2 stages x 64 KB
