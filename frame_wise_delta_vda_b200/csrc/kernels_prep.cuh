@@ -50,21 +50,23 @@ __host__ __device__ constexpr int kv_cols_per_thread(int Wl, int D) { return (Wl
 __host__ __device__ constexpr size_t kv_stage_bytes(int Wl, int D) {
   return (size_t)5 * (kv_slices(D) * kv_cols_per_thread(Wl, D) + 4) * D * 2;
 }
-// Shared memory: nst staging buffers of rows y-2..y+2 (bf16 pairs), the ring
-// of the last five frames' spatial results (bf16 pairs) and the fp32 output
-// row of the L2 normalisation.
+// Shared memory: nst staging buffers of rows y-2..y+2 (bf16 pairs), the
+// head's spatial filter taps (fp32, [25][d]) and the fp32 output row of the
+// L2 normalisation.
 __host__ __device__ constexpr size_t kv_smem_bytes(int Wl, int D, int nst) {
-  return (size_t)nst * kv_stage_bytes(Wl, D) + (size_t)5 * Wl * D * 2 + (size_t)Wl * D * 4;
+  return (size_t)nst * kv_stage_bytes(Wl, D) + (size_t)25 * D * 4 + (size_t)Wl * D * 4;
 }
 
 // One CTA per (grid row y, batch-head, tensor K or V).  It walks the frames:
 // the rows y-2..y+2 of a frame arrive by cp.async one frame ahead (two
 // staging buffers when they fit, else one, refilled once the spatial filter
-// has read it); the spatial filter of row y goes into a five-frame ring, and,
-// two frames behind, the temporal filter, SiLU and (K only) the L2
-// normalisation of output frame t.  Thread = (channel pair cp, column slice
-// xs): channel pairs use packed fp32 FMAs, and each thread keeps its NXT
-// columns' accumulators and the 5-tap window of one staged row in registers.
+// has read it).  Thread = (channel pair cp, column slice xs): it computes the
+// spatial 5 x 5 filter of row y for its NXT columns with packed fp32 FMAs and
+// a register window, and, since the same thread produces every frame of its
+// columns, it keeps the temporal filter's five running sums in registers:
+// frame f adds tap 4 - j to the sum of output frame f - 2 + j, and output
+// frame f - 2 is complete after frame f (then SiLU, and for K the L2
+// normalisation over the token's channels, one warp per token).
 template <int D, int NXT>
 __global__ void __launch_bounds__(kThreads, 1)
 k_prep_kv(const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict__ vin,
@@ -78,9 +80,9 @@ k_prep_kv(const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict
   constexpr int V8 = D / 8;              // 16-B chunks per token
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const size_t stage_words = (size_t)5 * WS * NP;
-  uint32_t* stage0 = reinterpret_cast<uint32_t*>(smem_raw);                  // [nst][5][WS][NP]
-  uint32_t* ring = stage0 + (size_t)nst * stage_words;                       // [5][Wl][NP]
-  float* tile = reinterpret_cast<float*>(ring + (size_t)5 * Wl * NP);        // [Wl][D]
+  uint32_t* stage0 = reinterpret_cast<uint32_t*>(smem_raw);                        // [nst][5][WS][NP]
+  float2* wsm = reinterpret_cast<float2*>(stage0 + (size_t)nst * stage_words);    // [25][NP]
+  float* tile = reinterpret_cast<float*>(wsm + (size_t)25 * NP);                 // [Wl][D]
 
   const int y = blockIdx.x, bh = blockIdx.y, isv = blockIdx.z;
   const int b = bh / H, h = bh - (bh / H) * H;
@@ -93,12 +95,14 @@ k_prep_kv(const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict
   const int c0 = 2 * cp;
   const int xb = xs * NXT;
 
-  float2 wsp[25], wtp[5];
-#pragma unroll
-  for (int q = 0; q < 25; ++q) wsp[q] = make_float2(__ldg(ws + (size_t)c0 * 25 + q), __ldg(ws + (size_t)(c0 + 1) * 25 + q));
+  float2 wtp[5];
 #pragma unroll
   for (int s = 0; s < 5; ++s) wtp[s] = make_float2(__ldg(wt + (size_t)c0 * 5 + s), __ldg(wt + (size_t)(c0 + 1) * 5 + s));
-
+  // the spatial taps of this head, [tap][channel pair]
+  for (int e = tid; e < 25 * NP; e += kThreads) {
+    const int q = e / NP, p2 = e - q * NP;
+    wsm[e] = make_float2(__ldg(ws + (size_t)(2 * p2) * 25 + q), __ldg(ws + (size_t)(2 * p2 + 1) * 25 + q));
+  }
   // padding columns and rows outside the grid are never loaded: zero them once
   for (size_t e = tid; e < (size_t)nst * stage_words; e += kThreads) stage0[e] = 0u;
   __syncthreads();
@@ -121,15 +125,17 @@ k_prep_kv(const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict
     cp_async_commit();
   };
   issue(0);
-  if (nst == 2 && T > 1) issue(1);
+
+  float2 tacc[5][NXT];   // running sums of output frames f - 2 .. f + 2
+#pragma unroll
+  for (int j = 0; j < 5; ++j)
+#pragma unroll
+    for (int i = 0; i < NXT; ++i) tacc[j][i] = make_float2(0.f, 0.f);
 
   for (int f = 0; f < T + 2; ++f) {
-    if (f < T) {   // this frame's rows have landed (the next frame's may still be in flight)
-      if (nst == 2 && f + 1 < T) cp_async_wait<1>();
-      else cp_async_wait<0>();
-    }
-    __syncthreads();   // ... for every thread; the previous frame's ring and tile reads are done
-    uint32_t* ring_t = ring + (size_t)(f % 5) * Wl * NP;
+    if (f < T) cp_async_wait<0>();   // this frame's rows have landed (this thread's copies)
+    __syncthreads();   // ... every thread's; the previous frame's staging and tile reads are done
+    if (nst == 2 && f + 1 < T) issue(f + 1);   // into the buffer frame f - 1 used
     if (f < T) {
       const uint32_t* st = stage0 + (size_t)(f % nst) * stage_words + cp;
       float2 acc[NXT];
@@ -139,6 +145,9 @@ k_prep_kv(const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict
       for (int dy = 0; dy < 5; ++dy) {
         const int row = y + dy - 2;
         if (row < 0 || row >= Hl) continue;   // a zero row
+        float2 w5[5];
+#pragma unroll
+        for (int dx = 0; dx < 5; ++dx) w5[dx] = wsm[(dy * 5 + dx) * NP + cp];
         const uint32_t* srow = st + (size_t)dy * WS * NP + (size_t)xb * NP;
         float2 win[NXT + 4];
 #pragma unroll
@@ -147,45 +156,45 @@ k_prep_kv(const __nv_bfloat16* __restrict__ kin, const __nv_bfloat16* __restrict
         for (int i = 0; i < NXT; ++i) {
           float2 a = acc[i];
 #pragma unroll
-          for (int dx = 0; dx < 5; ++dx) a = ffma2(wsp[dy * 5 + dx], win[i + dx], a);
+          for (int dx = 0; dx < 5; ++dx) a = ffma2(w5[dx], win[i + dx], a);
           acc[i] = a;
         }
       }
+      // frame f is tap 4 - j of output frame f - 2 + j
 #pragma unroll
-      for (int i = 0; i < NXT; ++i)
-        if (xb + i < Wl) ring_t[(size_t)(xb + i) * NP + cp] = f2_to_bf2(acc[i]);
-    } else {
-      // frames past the clip contribute zero (temporal zero padding)
+      for (int j = 0; j < 5; ++j)
 #pragma unroll
-      for (int i = 0; i < NXT; ++i)
-        if (xb + i < Wl) ring_t[(size_t)(xb + i) * NP + cp] = 0u;
-    }
-    __syncthreads();   // ring slot written; this frame's staging buffer has been read
-    if (f + nst < T) issue(f + nst);
-    if (f < 2) continue;
-    // temporal filter, SiLU of output frame tout = f - 2
-    const int tout = f - 2;
-#pragma unroll
-    for (int i = 0; i < NXT; ++i) {
-      const int x = xb + i;
-      if (x >= Wl) continue;
-      float2 o = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int s = 0; s < 5; ++s) {
-        const int fr = tout + s - 2;
-        if (fr < 0) continue;   // frames before the clip: zero padding
-        o = ffma2(wtp[s], bf2_to_f2(ring[((size_t)(fr % 5) * Wl + x) * NP + cp]), o);
-      }
-      o.x = silu(o.x);
-      o.y = silu(o.y);
-      if (isv) {
-        const size_t orow = (((size_t)bh * T + tout) * U + (size_t)y * Wl + x) * D;
-        reinterpret_cast<uint32_t*>(out + orow)[cp] = f2_to_bf2(o);
-      } else {
-        reinterpret_cast<float2*>(tile + (size_t)x * D)[cp] = o;
+        for (int i = 0; i < NXT; ++i) tacc[j][i] = ffma2(wtp[4 - j], acc[i], tacc[j][i]);
+      if (nst == 1) {   // refill the only staging buffer once every thread has read it
+        __syncthreads();
+        if (f + 1 < T) issue(f + 1);
       }
     }
-    if (!isv) {   // L2 normalisation of each token of the row, one warp per token
+    if (f >= 2) {   // output frame tout = f - 2 is complete: SiLU
+      const int tout = f - 2;
+#pragma unroll
+      for (int i = 0; i < NXT; ++i) {
+        const int x = xb + i;
+        if (x >= Wl) continue;
+        float2 o = tacc[0][i];
+        o.x = silu(o.x);
+        o.y = silu(o.y);
+        if (isv) {
+          const size_t orow = (((size_t)bh * T + tout) * U + (size_t)y * Wl + x) * D;
+          reinterpret_cast<uint32_t*>(out + orow)[cp] = f2_to_bf2(o);
+        } else {
+          reinterpret_cast<float2*>(tile + (size_t)x * D)[cp] = o;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < NXT; ++i) tacc[j][i] = tacc[j + 1][i];
+#pragma unroll
+    for (int i = 0; i < NXT; ++i) tacc[4][i] = make_float2(0.f, 0.f);
+    if (!isv && f >= 2) {   // L2 normalisation of each token of the row, one warp per token
+      const int tout = f - 2;
       __syncthreads();
       const int warp = tid >> 5, lane = tid & 31;
       constexpr int PER = D / 32 > 0 ? D / 32 : 1;

@@ -250,10 +250,10 @@ VDA_API int vda_launches_per_forward(int B, int H, int T, int U, int d_k, int d_
  *   wk_s, wv_s        [H, d, 5, 5] float32, wk_t, wv_t [H, d, 5] float32
  *   q_out, k_out, v_out [B, H, T, U, d] bf16 (the layout vda_forward reads)
  * Supported: bf16, d in {16, 32, 64, 128}, at most 8 grid columns per
- * thread slice (Wl <= 8 * 1024 / d) and the staging rows, the five-frame ring
- * and one fp32 output row (about (5 (Wl + 4) + 5 Wl + 2 Wl) * 2 d bytes)
- * within the device's shared memory (Wl <= 64 at d = 128).  Inputs and
- * outputs must not overlap.
+ * thread slice (Wl <= 8 * 1024 / d) and the staged rows, the spatial taps and
+ * one fp32 output row (about 5 (Wl + 4) * 2 d + 100 d + 4 d Wl bytes) within
+ * the device's shared memory (Wl <= 64 at d = 128).  Inputs and outputs must
+ * not overlap.
  * Returns vda_status. */
 typedef struct vda_prep_args {
   const void* q_in;
