@@ -113,6 +113,24 @@ def test_launch_count(L):
     assert L.vda_launches_per_forward(1, 6, 60, 1008, 128, 128, 1, 0) == 4   # one-frame chunks
 
 
+@pytest.mark.parametrize("H,chunk,T,launches", [
+    (6, 5, 60, 5),    # six heads: 288 composition CTAs, two waves
+    (7, 5, 60, 4), (12, 5, 60, 4), (24, 5, 60, 4), (48, 5, 60, 4),
+    (16, 5, 30, 4),   # the correlated-key shapes: 384 CTAs
+    (2, 5, 30, 5),
+    (6, 5, 5, 4),     # a single chunk: nothing to shorten
+    (2, 1, 60, 4),    # one-frame chunks: nothing to compose
+])
+def test_automatic_scan_form(L, H, chunk, T, launches):
+    # the chunk-wise scans (two launches) when their 4 B H NC composition CTAs
+    # fit in two waves of 148 SMs, with more than one frame per chunk and more
+    # than one chunk; otherwise the per-frame scans (one launch)
+    nc = (T + chunk - 1) // chunk
+    rule = 5 if (chunk > 1 and T > chunk and 4 * H * nc <= 2 * 148) else 4
+    assert launches == rule
+    assert L.vda_launches_per_forward(1, H, T, 256, 128, 128, chunk, 0) == launches
+
+
 def test_d64_tensor_core_workspace(L):
     # d = 64, bf16: the tensor-core path adds the scan's operand images
     # (16 KB per frame-head) to A/M, B and the boundary states; fp32 I/O at
