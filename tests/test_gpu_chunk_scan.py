@@ -90,6 +90,7 @@ EDGE = [
     ("chunk3_w0", dict(H=3, T=10, U=33, chunk=3, window_chunks=0)),
     ("decay_ragged", dict(H=2, T=11, U=64, chunk=4, window_chunks=1, alpha_mean=1.5)),
     ("decay_T1", dict(H=1, T=1, U=64, chunk=5, window_chunks=0, alpha_mean=1.5)),
+    ("B2", dict(B=2, H=2, T=12, U=48, chunk=4, window_chunks=1)),
 ]
 
 

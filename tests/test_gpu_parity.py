@@ -123,6 +123,7 @@ EDGE = [
     ("B2_d64", dict(B=2, H=3, T=10, U=33, d=64, chunk=5, window_chunks=1, dtype="f32")),
     ("d128_f32", dict(H=2, T=10, U=70, d=128, chunk=5, window_chunks=1, dtype="f32")),
     ("bf16_d64_ragged", dict(H=2, T=13, U=40, d=64, chunk=5, window_chunks=1, dtype="bf16")),
+    ("bf16_d64_B2", dict(B=2, H=3, T=9, U=70, d=64, chunk=4, window_chunks=1, dtype="bf16")),
     ("bf16_d128_oddU", dict(H=2, T=11, U=129, d=128, chunk=5, window_chunks=1, dtype="bf16")),
     ("bf16_d128_U1", dict(H=1, T=6, U=1, d=128, chunk=2, window_chunks=0, dtype="bf16")),
     ("bf16_d128_long_chunk", dict(H=1, T=4, U=300, d=128, chunk=3, window_chunks=0, dtype="bf16")),
