@@ -34,9 +34,24 @@ def test_status_strings(L):
 def test_status_enum_matches_header():
     text = open(_lib.HEADER).read()
     for name in ("VDA_OK", "VDA_ERR_INVALID_ARGUMENT", "VDA_ERR_UNSUPPORTED", "VDA_ERR_WORKSPACE",
-                 "VDA_ERR_CUDA", "VDA_ERR_TIMEOUT", "VDA_BF16", "VDA_F32"):
+                 "VDA_ERR_CUDA", "VDA_ERR_TIMEOUT", "VDA_BF16", "VDA_F32", "VDA_SCAN_AUTO", "VDA_SCAN_FRAMES",
+                 "VDA_SCAN_CHUNKS"):
         m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
         assert m and int(m.group(1)) == getattr(_lib, name), name
+
+
+@pytest.mark.parametrize("struct,mirror", [("vda_args", VdaArgs), ("vda_prep_args", _lib.VdaPrepArgs)])
+def test_argument_structs_mirror_the_header(struct, mirror):
+    """The ctypes mirrors list the C structs' fields in the header's order."""
+    text = open(_lib.HEADER).read()
+    body = re.search(r"typedef struct " + struct + r" \{(.*?)\} " + struct + ";", text, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if decl:
+            fields += [n.strip().lstrip("*") for n in re.sub(r"^(const\s+)?\w+\s*\**", "", decl).split(",")]
+    assert fields == [f[0] for f in mirror._fields_]
 
 
 def test_workspace_bytes(L):
