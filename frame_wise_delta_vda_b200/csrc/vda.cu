@@ -220,6 +220,10 @@ int validate_args(const vda_args* a) {
       (a->alpha && !aligned16(a->alpha)))
     return VDA_ERR_INVALID_ARGUMENT;
   if (a->scan_form < VDA_SCAN_AUTO || a->scan_form > VDA_SCAN_CHUNKS) return VDA_ERR_INVALID_ARGUMENT;
+  // the chunk-wise scans launch one CTA per (b, h, chunk, direction, part)
+  if (a->scan_form == VDA_SCAN_CHUNKS &&
+      4.0 * a->B * a->H * (double)((a->T + a->chunk - 1) / a->chunk) > 2147483647.0)
+    return VDA_ERR_UNSUPPORTED;
   return VDA_OK;
 }
 

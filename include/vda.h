@@ -94,7 +94,9 @@ typedef enum vda_dtype {
  *     into one affine map S -> S P_c + J_c, then each chain runs its NC maps.
  *     About twice the tensor-core work on a chain of chunk + NC steps; it pays
  *     when few (b, h) pairs share the GPU.
- *   VDA_SCAN_AUTO: the library picks by the number of (b, h) pairs. */
+ *   VDA_SCAN_AUTO: the library picks by the number of (b, h) pairs.
+ * VDA_SCAN_CHUNKS with more than 2^31 - 1 composition CTAs (4 B H NC) returns
+ * VDA_ERR_UNSUPPORTED. */
 typedef enum vda_scan_form {
   VDA_SCAN_AUTO = 0,
   VDA_SCAN_FRAMES = 1,

@@ -90,6 +90,7 @@ def _args(**kw):
     (dict(d_k=16, d_v=32), 2),             # d_k != d_v
     (dict(d_k=48, d_v=48), 2),             # unsupported head dim
     (dict(scan_form=3), 1), (dict(scan_form=-1), 1),
+    (dict(scan_form=2, H=800000, T=1500, chunk=2), 2),   # 4 x 800000 x 750 composition CTAs
 ])
 def test_forward_ex_rejects_bad_arguments(L, kw, status):
     a = _args(**kw)
